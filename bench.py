@@ -1,0 +1,431 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 SmoothQuant W8A8 INT8 linear layer.
+
+One step = one pass of the layer's hot path over one batch: per-token
+dynamic INT8 quantisation of X with the SmoothQuant 1/s fold, then the
+INT8 x INT8 GEMM with the fused per-token x per-channel BF16 epilogue, on the
+prefill workload M=8192 tokens, K=5120, N=34816 (fused gate/up shape).
+The printed metric is TOPS (2*M*N*K per step, quantisation included in the
+time).  The same run also measures the decode W8A8 shape, the gs128
+variant and the W8A16 (down_proj) variant at M = 1, 16, 8192.
+
+  python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+
+N > 1 (under torchrun) runs N independent replicas of the same workload,
+one per GPU (the layer has no exchange step on one GPU); value is the sum
+of the work over the max of the per-rank device times.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+METRIC = "W8A8 GEMM TOPS incl. per-token quant (% of INT8 peak); W8A16 GB/s at M≤16"
+INT8_PER_BF16 = 2.0          # dense INT8 ops per dense BF16 flop (4.5 / 2.25 PFLOP/s nominal)
+INT8_NOMINAL_TOPS = 4500.0   # dense INT8, nominal B200
+
+
+def load_peaks():
+    try:
+        d = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+# ------------------------------------------------------------- clock sampler
+class ClockSampler(threading.Thread):
+    """Samples the SM clock and clock-event reasons through NVML every 5 ms."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, device: int):
+        super().__init__(daemon=True)
+        self.samples = []
+        self.reasons = 0
+        self.stop_evt = threading.Event()
+        self.ok = False
+        self.max_mhz = None
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            self.nv = nv
+            self.h = self._handle(device)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM)
+            self.get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons")
+            self.ok = True
+        except Exception:
+            self.ok = False
+
+    def _handle(self, device):
+        nv = self.nv
+        try:
+            p = torch.cuda.get_device_properties(device)
+            bus = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+            return nv.nvmlDeviceGetHandleByPciBusId(bus.encode())
+        except Exception:
+            return nv.nvmlDeviceGetHandleByIndex(0)
+
+    def run(self):
+        if not self.ok:
+            return
+        nv = self.nv
+        while not self.stop_evt.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                self.reasons |= int(self.get_reasons(self.h))
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def result(self):
+        self.stop_evt.set()
+        self.join(timeout=2)
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        busy = [s for s in self.samples if s > 0]
+        return {"sm_mhz": statistics.median(busy or self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": [n for b, n in self.REASONS.items() if self.reasons & b and b != 0x1],
+                "samples": len(self.samples)}
+
+
+# -------------------------------------------------------------------- helpers
+def algo_bytes_quant(M, K):
+    return 2 * M * K + 4 * K + M * K + 4 * M
+
+
+def algo_bytes_w8a8(M, N, K, gs=False):
+    scales = 4 * N * (K // 128) if gs else 4 * N
+    return M * K + N * K + 4 * M + scales + 2 * M * N
+
+
+def algo_bytes_w8a16(M, N, K):
+    return 2 * M * K + N * K + 4 * N + 2 * M * N
+
+
+def time_batches(fn, iters, warmup=3):
+    """Device time per call of fn (back-to-back launches on the current stream)."""
+    for i in range(warmup):
+        fn(i)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for i in range(iters):
+        fn(i)
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / iters * 1e-3
+
+
+def dist_info():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+# ------------------------------------------------------------ CPU oracle leg
+def oracle_sample(wl, target_s: float, max_rows: int = None):
+    """Times the CPU oracle (quant + W8A8 GEMM) on a bounded row sample."""
+    import oracle
+    x = wl.make_x()
+    w = wl.make_w()
+    s, inv = oracle.smooth_factors(x, w)
+    q_w, s_ch = oracle.quant_weight(w, s)
+    del w
+    nt = oracle.threads()
+
+    def run(rows):
+        xs = x[:rows].contiguous()
+        t0 = time.perf_counter()
+        q_a, s_tok = oracle.quant_per_token(xs, inv)
+        oracle.w8a8_scaled_mm(q_a, s_tok, q_w, s_ch)
+        return time.perf_counter() - t0
+
+    t1 = run(nt)
+    rows = max(1, min(wl.M, int(nt * target_s / max(t1, 1e-6))))
+    if max_rows:
+        rows = min(rows, max_rows)
+    return rows, nt, run
+
+
+def reference_arm(args, peaks):
+    ws, rank, _ = dist_info()
+    if rank != 0:
+        return 0
+    from w8a8_int8_quantized_sq_b200 import inputs
+    wl = inputs.workload(2)
+    rows, nt, run = oracle_sample(wl, target_s=0.5)
+    ops_step = 2.0 * rows * wl.N * wl.K
+    for _ in range(args.warmup):
+        run(rows)
+    t = 0.0
+    for _ in range(args.steps):
+        t += run(rows)
+    value = ops_step * args.steps / t / 1e12
+    sample = (f"first {rows} of {wl.M} token rows of {wl.name} per step "
+              "(oracle per-token quant + int32 GEMM + epilogue, all N columns)")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TOPS",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": t / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+            "config": {"workload": wl.name, "M": wl.M, "K": wl.K, "N": wl.N,
+                       "rows_per_step": rows},
+            "cpu_baseline": {"value": value, "unit": "TOPS", "cores": nt, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------- main arm
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-variants", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    peaks = load_peaks()
+    if args.impl == "reference":
+        return reference_arm(args, peaks)
+
+    import w8a8_int8_quantized_sq_b200 as sq
+    from w8a8_int8_quantized_sq_b200 import inputs
+
+    world, rank, local = dist_info()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    sq.lib()  # fails loudly if the CUDA library is missing
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        return float(t.item())
+
+    # ---------------- prefill W8A8 (the headline workload)
+    wl = inputs.workload(2)
+    M, N, K = wl.M, wl.N, wl.K
+    x_cpu = wl.make_x()
+    x = x_cpu.to(dev)
+    w = wl.make_w().to(dev)
+    s_sm, inv_s = sq.smooth_factors(x, w)
+    q_w, s_ch = sq.quant_weight(w, s_sm)
+    del w
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    torch.cuda.synchronize()
+
+    def step():
+        q_a, s_tok = sq.quant_per_token(x, inv_s)
+        sq.w8a8_scaled_mm(q_a, s_tok, q_w, s_ch, out=y)
+        return q_a, s_tok
+
+    for _ in range(args.warmup):
+        step()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    barrier()
+    sampler.start()
+    start.record()
+    for i in range(args.steps):
+        ev[i][0].record()
+        q_a, s_tok = sq.quant_per_token(x, inv_s)
+        ev[i][1].record()
+        sq.w8a8_scaled_mm(q_a, s_tok, q_w, s_ch, out=y)
+        ev[i][2].record()
+    end.record()
+    barrier()
+    clocks = sampler.result()
+    total_s = max_over_ranks(start.elapsed_time(end) * 1e-3)
+    quant_s = statistics.mean(e[0].elapsed_time(e[1]) for e in ev) * 1e-3
+    gemm_s = statistics.mean(e[1].elapsed_time(e[2]) for e in ev) * 1e-3
+    ops_step = 2.0 * M * N * K
+    value = ops_step * args.steps * world / total_s / 1e12
+    int8_peak = peaks["bf16_tflops"] * INT8_PER_BF16
+    gemm_tops = ops_step / gemm_s / 1e12
+
+    # ---------------- end to end through the public API, host buffers
+    e2e_steps = max(3, min(args.steps, 10))
+    x_h = x_cpu.pin_memory()
+    y_h = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    x_d = torch.empty_like(x)
+
+    def e2e_step():
+        x_d.copy_(x_h, non_blocking=True)
+        yy = sq.linear_w8a8(x_d, inv_s, q_w, s_ch)
+        y_h.copy_(yy, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(e2e_steps):
+        e2e_step()
+    b.record()
+    barrier()
+    e2e_s = max_over_ranks(a.elapsed_time(b) * 1e-3)
+    e2e = {"value": ops_step * e2e_steps * world / e2e_s / 1e12, "unit": "TOPS",
+           "h2d_bytes_per_step": x_h.numel() * 2, "d2h_bytes_per_step": y_h.numel() * 2,
+           "steps": e2e_steps}
+    del x_h, y_h, x_d
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": total_s / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+        "config": {"workload": wl.name, "M": M, "K": K, "N": N,
+                   "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": "inputs larger than L2 (q_w 178 MB, x 84 MB, y 570 MB)",
+                   "step": "sq_quant_per_token + w8a8_scaled_mm"},
+        "pct_of_int8_nominal": 100.0 * value / world / INT8_NOMINAL_TOPS,
+        "roofline": {"bound": "tensor", "kernel": "gemm_kernel (W8A8, 128x256 tiles)",
+                     "achieved": gemm_tops, "peak": int8_peak, "unit": "TOPS",
+                     "frac": gemm_tops / int8_peak,
+                     "peak_source": f"{peaks['source']} bf16 burst x {INT8_PER_BF16:g}",
+                     "traffic": None},
+        "split_ms": {"quant": quant_s * 1e3, "gemm": gemm_s * 1e3},
+        "quant_hbm": {"achieved_gbs": algo_bytes_quant(M, K) / quant_s / 1e9,
+                      "peak_gbs": peaks["hbm_gbs"],
+                      "frac": algo_bytes_quant(M, K) / quant_s / 1e9 / peaks["hbm_gbs"]},
+        "e2e": e2e,
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks,
+    }
+    del x, q_w, y
+    torch.cuda.empty_cache()
+
+    if not args.no_variants:
+        line["variants"] = variants(sq, inputs, dev, peaks)
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rows, nt, run = oracle_sample(wl, target_s=args.cpu_seconds)
+        t = run(rows)
+        line["cpu_baseline"] = {
+            "value": 2.0 * rows * N * K / t / 1e12, "unit": "TOPS", "cores": nt,
+            "kind": "oracle", "seconds": t,
+            "sample": f"first {rows} of {M} token rows of {wl.name} (oracle quant + GEMM + "
+                      "epilogue over all N columns)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def variants(sq, inputs, dev, peaks):
+    """The other workloads, each timed alone with enough weight copies to exceed L2."""
+    out = []
+    hbm = peaks["hbm_gbs"]
+    l2 = 126 * 2 ** 20
+
+    # decode-shaped W8A8 (M=8): weight-read bound
+    wl = inputs.workload(1)
+    x = wl.make_x().to(dev)
+    w = wl.make_w().to(dev)
+    s, inv = sq.smooth_factors(x, w)
+    q_w, s_ch = sq.quant_weight(w, s)
+    del w
+    copies = max(2, -(-3 * l2 // q_w.numel()))
+    qws = [q_w.clone() for _ in range(copies)]
+    t = time_batches(lambda i: sq.linear_w8a8(x, inv, qws[i % copies], s_ch), 60)
+    tg = time_batches(lambda i: sq.w8a8_scaled_mm(*sq.quant_per_token(x, inv), qws[i % copies],
+                                                  s_ch), 60)
+    byt = algo_bytes_quant(wl.M, wl.K) + algo_bytes_w8a8(wl.M, wl.N, wl.K)
+    out.append({"workload": wl.name, "metric": "GB/s (quant + GEMM, algorithmic bytes)",
+                "value": byt / t / 1e9, "unit": "GB/s", "us_per_call": t * 1e6,
+                "frac_of_hbm": byt / t / 1e9 / hbm, "tokens_per_s": wl.M / t,
+                "tops": 2.0 * wl.M * wl.N * wl.K / t / 1e12, "weight_copies": copies,
+                "us_per_call_recheck": tg * 1e6})
+    del qws, q_w, x
+
+    # gs128 W8A8 (M=2048)
+    wl = inputs.workload(3)
+    x = wl.make_x().to(dev)
+    w = wl.make_w().to(dev)
+    q_w, s_blk = sq.quant_weight(w, None, group=128)
+    del w
+    q_a, s_tok = sq.quant_per_token(x, None)
+    copies = max(2, -(-3 * l2 // (q_w.numel() + q_a.numel())))
+    sets = [(q_a.clone(), q_w.clone()) for _ in range(copies)]
+    t = time_batches(lambda i: sq.w8a8_gs128_mm(sets[i % copies][0], s_tok, sets[i % copies][1],
+                                                s_blk), 30)
+    tq = time_batches(lambda i: sq.quant_per_token(x, None), 30)
+    ops = 2.0 * wl.M * wl.N * wl.K
+    int8_peak = peaks["bf16_tflops"] * INT8_PER_BF16
+    out.append({"workload": wl.name, "metric": "TOPS (gs128 GEMM)", "value": ops / t / 1e12,
+                "unit": "TOPS", "us_per_call": t * 1e6, "frac_of_int8_peak": ops / t / 1e12 / int8_peak,
+                "tops_incl_quant": ops / (t + tq) / 1e12, "quant_us": tq * 1e6,
+                "weight_copies": copies})
+    del sets, q_w, q_a, x
+
+    # W8A16 down_proj (K=17408, N=5120), M = 1, 16, 8192
+    wl = inputs.workload(4)
+    w = wl.make_w().to(dev)
+    q_w, s_ch = sq.quant_weight(w, None)
+    del w
+    copies = max(2, -(-3 * l2 // q_w.numel()))
+    qws = [q_w] + [q_w.clone() for _ in range(copies - 1)]
+    for M in inputs.W8A16_M_VALUES:
+        x = wl.make_x(M).to(dev)
+        if M <= 16:
+            t = time_batches(lambda i: sq.w8a16_mm(x, qws[i % copies], s_ch), 60)
+            byt = algo_bytes_w8a16(M, wl.N, wl.K)
+            out.append({"workload": f"{wl.name}_M{M}", "metric": "GB/s (algorithmic bytes)",
+                        "value": byt / t / 1e9, "unit": "GB/s", "us_per_call": t * 1e6,
+                        "frac_of_hbm": byt / t / 1e9 / hbm, "tokens_per_s": M / t,
+                        "weight_copies": copies})
+        else:
+            t = time_batches(lambda i: sq.w8a16_mm(x, qws[i % 2], s_ch), 10)
+            fl = 2.0 * M * wl.N * wl.K
+            out.append({"workload": f"{wl.name}_M{M}", "metric": "TFLOP/s (bf16 tensor)",
+                        "value": fl / t / 1e12, "unit": "TFLOP/s", "us_per_call": t * 1e6,
+                        "frac_of_bf16_peak": fl / t / 1e12 / peaks["bf16_tflops"],
+                        "tokens_per_s": M / t})
+        del x
+    del qws, q_w
+    torch.cuda.empty_cache()
+    return out
+
+
+if __name__ == "__main__":
+    sys.exit(main())

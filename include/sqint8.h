@@ -1,0 +1,139 @@
+/*
+ * sqint8.h -- C ABI of the B200 (sm_100a) SmoothQuant W8A8 INT8 linear layer.
+ *
+ * Every call is asynchronous on the caller's CUDA stream (passed as a
+ * cudaStream_t cast to void*; NULL is the legacy default stream).  The
+ * library never allocates device memory and never synchronises: the caller
+ * owns every buffer (device pointers, row-major, contiguous, 16-byte
+ * aligned) and the stream.  Errors are returned as sq_status; nothing aborts,
+ * exits or traps.  A kernel wait that exceeds its time limit makes the kernel
+ * return early and latch a device error word, read by sq_check_device_error.
+ *
+ * Shapes: M >= 0 tokens, N > 0 output channels with N % 16 == 0,
+ * K > 0 input channels with K % 128 == 0 and K <= 131072 (so that
+ * K * 127 * 127 fits in int32).  M == 0 is a no-op.
+ *
+ * Sources (page title, section):
+ *  [P1] "Qwen3.8-27B - SmoothQuant + activation-aware GPTQ, W8A8 INT8 (v3)",
+ *       "Recipe" items 1-2 and "Serving": SmoothQuant folds; INT8 per-channel
+ *       symmetric weights with INT8 per-token dynamic activations (W8A8) on
+ *       a scaled-mm kernel; INT8 per-channel weights with BF16 activations
+ *       (W8A16) for down_proj on a weight-only dequant kernel.
+ *  [P2] "lued/Qwen3.8-27B-INT8-W8A16-MTP", "Why W8A16 on Ampere": weight-only
+ *       kernels reconstruct the weights for 16-bit GEMMs.
+ *  [P3] "Qwen3.8-27B - FP8 block + AWQ", "Recipe" item 1: 1/s folds into the
+ *       preceding op, s into the next linear's input dimension.
+ *  [P4] "Qwen3.8-27B-INT8-W8A8", "Quantization": symmetric per-output-channel
+ *       INT8 weights, dynamic per-token INT8 activations.
+ *  [P5] "Qwen3.8-27B-GPTQ-INT8-W8A8-GS128", "Quantization details" and
+ *       "Why group_size 128": one weight scale per 128-wide K block with INT8
+ *       x INT8 compute and dynamically quantised inputs.
+ */
+#ifndef SQINT8_H
+#define SQINT8_H
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SQ_OK = 0,
+  SQ_ERR_NULL = 1,        /* a required pointer is NULL                          */
+  SQ_ERR_SHAPE = 2,       /* a size breaks the rules above                       */
+  SQ_ERR_ALIGN = 3,       /* a pointer is not 16-byte aligned                    */
+  SQ_ERR_WORKSPACE = 4,   /* workspace missing or smaller than sq_workspace_bytes */
+  SQ_ERR_CUDA = 5,        /* a CUDA runtime/driver call failed                   */
+  SQ_ERR_TIMEOUT = 6      /* a kernel gave up a wait (sq_check_device_error)     */
+} sq_status;
+
+/* Operation ids for sq_workspace_bytes. */
+enum { SQ_OP_W8A8 = 0, SQ_OP_GS128 = 1, SQ_OP_W8A16 = 2, SQ_OP_W8A8_I32 = 3 };
+
+/* Per-token dynamic INT8 quantisation with the SmoothQuant 1/s fold [P1, P3, P4].
+ * For each row m of x (BF16 [M,K]):  x'[k] = f32(x[m,k]) * inv_smooth[k]
+ * (one fp32 rounding), amax = max_k |x'[k]|, s_tok[m] = amax / 127,
+ * q_i8[m,k] = clamp(rint(x'[k] * (127 / amax)), -127, 127) with
+ * round-half-even; an all-zero row gives s_tok = 0 and zero codes.
+ * inv_smooth (fp32 [K]) may be NULL (no smoothing).
+ * Outputs: q_i8 int8 [M,K], s_tok fp32 [M]. */
+sq_status sq_quant_per_token(const void* x_bf16, const float* inv_smooth, int8_t* q_i8,
+                             float* s_tok, int64_t M, int64_t K, void* stream);
+
+/* W8A8 INT8 GEMM with the fused per-token x per-channel dequant epilogue
+ * [P1 "Serving", P4]:  acc[m,n] = sum_k q_a[m,k] * q_w[n,k] (exact int32),
+ * y[m,n] = bf16_rne((f32(acc) * s_tok[m]) * s_ch[n]).
+ * q_a int8 [M,K], s_tok fp32 [M], q_w int8 [N,K] (nn.Linear layout, K-major),
+ * s_ch fp32 [N], y_bf16 [M,N].  Small M (<= 32) uses a split-K schedule
+ * whose partial sums live in the caller's workspace (size from
+ * sq_workspace_bytes(SQ_OP_W8A8, ...); pass NULL/0 when it is 0).
+ * Workspace rule for every operation: the first 64 KiB hold arrival
+ * counters that must be zero before the workspace is first used; every call
+ * that completes on the device leaves them zero, and nothing else is written
+ * there, so one workspace may serve calls of any operation and size in
+ * stream order.  Calls that may overlap on the device need separate
+ * workspaces.  After SQ_ERR_TIMEOUT, zero the counters again. */
+sq_status w8a8_scaled_mm(const int8_t* q_a, const float* s_tok, const int8_t* q_w,
+                         const float* s_ch, void* y_bf16, int64_t M, int64_t N, int64_t K,
+                         void* workspace, size_t ws_bytes, void* stream);
+
+/* W8A8 with group-size-128 weight scales [P5]: s_blk fp32 [N, K/128], one
+ * scale per (output row, 128-wide K block).  With P_kb[m,n] the exact int32
+ * partial over block kb:  acc = 0; for kb ascending:
+ * acc = fmaf(f32(P_kb), s_blk[n,kb], acc);  y = bf16_rne(acc * s_tok[m]).
+ * Workspace as for w8a8_scaled_mm (SQ_OP_GS128; currently always 0). */
+sq_status w8a8_gs128_mm(const int8_t* q_a, const float* s_tok, const int8_t* q_w,
+                        const float* s_blk, void* y_bf16, int64_t M, int64_t N, int64_t K,
+                        void* workspace, size_t ws_bytes, void* stream);
+
+/* W8A16 weight-only GEMM [P1 "Recipe" item 2, P2]: x BF16 [M,K], q_w int8
+ * [N,K], s_ch fp32 [N]; y = bf16_rne(s_ch[n] * sum_k x[m,k] * q_w[n,k]).
+ * The int8 -> bf16 weight conversion is exact and the scale is applied in
+ * the fp32 epilogue; products are exact and accumulate in fp32 (the order
+ * of the fp32 sum is the kernel's).  Workspace (SQ_OP_W8A16) holds split-K
+ * partials for small M and the converted BF16 weights for large M; the
+ * zero-fill rule of w8a8_scaled_mm applies. */
+sq_status w8a16_mm(const void* x_bf16, const int8_t* q_w, const float* s_ch, void* y_bf16,
+                   int64_t M, int64_t N, int64_t K, void* workspace, size_t ws_bytes,
+                   void* stream);
+
+/* Bytes of workspace an operation needs for these sizes (0 = none). */
+size_t sq_workspace_bytes(int op, int64_t M, int64_t N, int64_t K);
+
+/* Raw int32 accumulators of the W8A8 mainloop (same kernels, no epilogue):
+ * acc int32 [M,N] = q_a . q_w^T.  Workspace as for SQ_OP_W8A8_I32. */
+sq_status w8a8_mm_i32(const int8_t* q_a, const int8_t* q_w, int32_t* acc, int64_t M,
+                      int64_t N, int64_t K, void* workspace, size_t ws_bytes, void* stream);
+
+/* Offline preparation -------------------------------------------------- */
+
+/* SmoothQuant factors from calibration maxima [P1 "Recipe" item 1]:
+ * s_j = clamp(sqrt(max_m |x[m,j]|) / sqrt(max_n |w[n,j]|), floor_, cap)
+ * computed in fp64 (alpha = 1/2); a column with both maxima zero gets 1, one
+ * with only max|w| zero gets cap.  s_out[j] = f32(s_j),
+ * inv_s_out[j] = f32(1 / s_out[j]).  x BF16 [M,K], w BF16 [N,K]; M, N >= 1. */
+sq_status sq_smooth_factors(const void* x_bf16, int64_t M, const void* w_bf16, int64_t N,
+                            int64_t K, double cap, double floor_, float* s_out,
+                            float* inv_s_out, void* stream);
+
+/* Symmetric INT8 weight quantisation of the folded weight W'[n,k] =
+ * f32(w[n,k]) * smooth[k] [P1, P3, P4, P5]; smooth may be NULL.  group == 0:
+ * scales fp32 [N] (per output channel); group == 128: scales fp32 [N, K/128].
+ * Scale = amax/127, codes as in sq_quant_per_token. */
+sq_status sq_quant_weight(const void* w_bf16, const float* smooth, int8_t* q_w, float* scales,
+                          int64_t N, int64_t K, int64_t group, void* stream);
+
+/* Diagnostics ------------------------------------------------------------ */
+
+/* Synchronises the current device, then returns SQ_ERR_TIMEOUT if any kernel
+ * of this library latched a timeout since the last reset (reset != 0 clears
+ * the word), SQ_ERR_CUDA if the device reports an error, else SQ_OK. */
+sq_status sq_check_device_error(int reset);
+
+const char* sq_status_string(sq_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

@@ -1,0 +1,251 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Bar: bit-exact on INT8 codes, scales and int32 accumulators; bit-exact on the
+W8A8 and gs128 BF16 outputs (the kernels take the oracle's rounding steps in
+the same order, which is within the 1-ulp allowance); W8A16 within one BF16
+ulp plus the fp32 accumulation bound stated in test_w8a16_parity.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import w8a8_int8_quantized_sq_b200 as sq
+from w8a8_int8_quantized_sq_b200 import inputs
+from tests.prep import bf16_ulp, to_cuda, workload
+
+pytestmark = pytest.mark.gpu
+
+
+def _bits(t: torch.Tensor) -> torch.Tensor:
+    return t.cpu().view(torch.int16) if t.dtype == torch.bfloat16 else t.cpu()
+
+
+def assert_same(gpu: torch.Tensor, ref: torch.Tensor, what: str):
+    g, r = _bits(gpu), _bits(ref)
+    if not torch.equal(g, r):
+        bad = (g != r).nonzero()
+        raise AssertionError(f"{what}: {bad.shape[0]} of {r.numel()} differ; first at "
+                             f"{bad[0].tolist()}: gpu {gpu.cpu()[tuple(bad[0])]} "
+                             f"ref {ref[tuple(bad[0])]}")
+
+
+# ----------------------------------------------------------------- quant
+
+@pytest.mark.parametrize("cfg", [0, 1, 2, 3, 4])
+def test_quant_per_token_configs(cfg):
+    d = workload(cfg)
+    x = d["x"]
+    inv = d["inv_s"]
+    q_ref, s_ref = oracle.quant_per_token(x, inv)
+    q, s = sq.quant_per_token(x.cuda(), inv.cuda() if inv is not None else None)
+    assert_same(q, q_ref, "q_a")
+    assert_same(s, s_ref, "s_tok")
+
+
+@pytest.mark.parametrize("M,K", [(1, 128), (7, 384), (129, 256), (2048, 128), (3000, 17408)])
+def test_quant_per_token_edges(M, K):
+    x = inputs.gen_x(M, K, 99, inputs.XRecipe(col_count=3, col_factor=40.0, row_period=5,
+                                              row_width=1, row_factor=50.0))
+    x[M // 2] = 0  # an all-zero row
+    inv = torch.rand(K, dtype=torch.float32) + 0.25
+    q_ref, s_ref = oracle.quant_per_token(x, inv)
+    q, s = sq.quant_per_token(x.cuda(), inv.cuda())
+    assert_same(q, q_ref, "q_a")
+    assert_same(s, s_ref, "s_tok")
+
+
+def test_quant_exact_integer_rows():
+    ints = torch.randint(-127, 128, (64, 256))
+    ints[:, 3] = 127
+    x = ints.float().to(torch.bfloat16)
+    q, s = sq.quant_per_token(x.cuda())
+    assert torch.equal(q.cpu().long(), ints) and torch.all(s.cpu() == 1.0)
+
+
+# ------------------------------------------------------- offline preparation
+
+@pytest.mark.parametrize("cfg", [0, 1])
+def test_smooth_and_weight_quant(cfg):
+    d = workload(cfg)
+    s, inv = sq.smooth_factors(d["x"].cuda(), d["w"].cuda())
+    assert_same(s, d["s"], "s")
+    assert_same(inv, d["inv_s"], "inv_s")
+    q, sc = sq.quant_weight(d["w"].cuda(), s)
+    assert_same(q, d["q_w"], "q_w")
+    assert_same(sc, d["s_ch"], "s_ch")
+
+
+def test_weight_quant_gs128():
+    d = workload(3)
+    q, sb = sq.quant_weight(d["w"].cuda(), None, group=128)
+    assert_same(q, d["q_w"], "q_w gs128")
+    assert_same(sb, d["s_blk"], "s_blk")
+
+
+# ----------------------------------------------------------- W8A8 GEMM
+
+@pytest.mark.parametrize("cfg", [0, 1, 3])
+def test_mm_i32_configs(cfg):
+    d = workload(cfg)
+    ref = oracle.mm_i32(d["q_a"], d["q_w"])
+    acc = sq.w8a8_mm_i32(d["q_a"].cuda(), d["q_w"].cuda())
+    assert_same(acc, ref, "int32 acc")
+
+
+SHAPES = [(1, 16, 128), (7, 144, 384), (16, 128, 256), (17, 272, 640), (32, 128, 1280),
+          (33, 256, 256), (129, 400, 384), (300, 528, 1024), (256, 512, 5120)]
+
+
+@pytest.mark.parametrize("M,N,K", SHAPES)
+def test_mm_i32_and_scaled_shapes(M, N, K):
+    g = torch.Generator().manual_seed(M * 7 + N * 3 + K)
+    q_a = torch.randint(-127, 128, (M, K), generator=g, dtype=torch.int8)
+    q_w = torch.randint(-127, 128, (N, K), generator=g, dtype=torch.int8)
+    s_tok = torch.rand(M, generator=g) * 0.1 + 1e-3
+    s_ch = torch.rand(N, generator=g) * 1e-3 + 1e-5
+    acc = sq.w8a8_mm_i32(q_a.cuda(), q_w.cuda())
+    assert_same(acc, oracle.mm_i32(q_a, q_w), "int32 acc")
+    y = sq.w8a8_scaled_mm(q_a.cuda(), s_tok.cuda(), q_w.cuda(), s_ch.cuda())
+    assert_same(y, oracle.w8a8_scaled_mm(q_a, s_tok, q_w, s_ch), "y")
+
+
+def test_mm_extreme_magnitudes():
+    K = 17408
+    q_a = torch.full((3, K), 127, dtype=torch.int8)
+    q_a[1] = -127
+    q_a[2, ::2] = -127
+    q_w = torch.full((32, K), 127, dtype=torch.int8)
+    acc = sq.w8a8_mm_i32(q_a.cuda(), q_w.cuda())
+    assert_same(acc, oracle.mm_i32(q_a, q_w), "int32 acc extremes")
+
+
+@pytest.mark.parametrize("cfg", [0, 1])
+def test_w8a8_scaled_mm_configs(cfg):
+    d = workload(cfg)
+    ref = oracle.w8a8_scaled_mm(d["q_a"], d["s_tok"], d["q_w"], d["s_ch"])
+    c = to_cuda(d)
+    y = sq.w8a8_scaled_mm(c["q_a"], c["s_tok"], c["q_w"], c["s_ch"])
+    assert_same(y, ref, "y")
+    # the full layer (quant + GEMM) from the raw activations
+    y2 = sq.linear_w8a8(c["x"], c["inv_s"], c["q_w"], c["s_ch"])
+    assert_same(y2, ref, "y (linear)")
+    # repeated calls are identical (stream-K counters reset themselves)
+    y3 = sq.w8a8_scaled_mm(c["q_a"], c["s_tok"], c["q_w"], c["s_ch"])
+    assert_same(y3, ref, "y (repeat)")
+
+
+def test_w8a8_prefill_full_size_sampled_rows():
+    """M=8192, K=5120, N=34816: the whole GEMM on the GPU, oracle on sampled rows."""
+    d = workload(2)
+    c = to_cuda(d)
+    q_a, s_tok = sq.quant_per_token(c["x"], c["inv_s"])
+    assert_same(q_a, d["q_a"], "q_a")
+    assert_same(s_tok, d["s_tok"], "s_tok")
+    y = sq.w8a8_scaled_mm(c["q_a"], c["s_tok"], c["q_w"], c["s_ch"])
+    rows = sorted({0, 1, 2, 3, 4, 127, 128, 511, 512, 515, 4096, 8191} |
+                  set(np.random.default_rng(0).integers(0, 8192, 12).tolist()))
+    ref = oracle.w8a8_scaled_mm(d["q_a"], d["s_tok"], d["q_w"], d["s_ch"], rows=rows)
+    assert_same(y.cpu()[rows], ref, "y sampled rows")
+    # a column sample over every row too (catches errors in other row tiles)
+    cols = [0, 255, 256, 17407, 34815]
+    acc = oracle.mm_i32(d["q_a"], d["q_w"][cols].contiguous())
+    yc = oracle.epilogue_ch(acc, d["s_tok"], d["s_ch"][cols].contiguous())
+    assert_same(y.cpu()[:, cols].contiguous(), yc, "y sampled columns")
+
+
+# ---------------------------------------------------------------- gs128
+
+def test_gs128_config():
+    d = workload(3)
+    ref = oracle.gs128_mm(d["q_a"], d["s_tok"], d["q_w"], d["s_blk"])
+    c = to_cuda(d)
+    y = sq.w8a8_gs128_mm(c["q_a"], c["s_tok"], c["q_w"], c["s_blk"])
+    assert_same(y, ref, "y gs128")
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 128, 128), (100, 256, 1024), (130, 384, 17408)])
+def test_gs128_shapes(M, N, K):
+    g = torch.Generator().manual_seed(M + N + K)
+    q_a = torch.randint(-127, 128, (M, K), generator=g, dtype=torch.int8)
+    q_w = torch.randint(-127, 128, (N, K), generator=g, dtype=torch.int8)
+    s_tok = torch.rand(M, generator=g) * 0.1 + 1e-3
+    s_blk = torch.rand(N, K // 128, generator=g) * 1e-3 + 1e-5
+    y = sq.w8a8_gs128_mm(q_a.cuda(), s_tok.cuda(), q_w.cuda(), s_blk.cuda())
+    assert_same(y, oracle.gs128_mm(q_a, s_tok, q_w, s_blk), "y gs128")
+
+
+# ---------------------------------------------------------------- W8A16
+
+def _check_w8a16(x, q_w, s_ch, rows=None):
+    y = sq.w8a16_mm(x.cuda(), q_w.cuda(), s_ch.cuda()).cpu()
+    if rows is not None:
+        y = y[rows]
+    ref, mag = oracle.w8a16_mm(x, q_w, s_ch, rows=rows, with_bound=True)
+    K = x.shape[1]
+    # fp32 accumulation: at most K/16 tensor-core steps plus the split-K
+    # combination, each adding at most 2^-22 of the magnitude sum.
+    gamma = (K / 16 + 8) * 2.0 ** -22
+    diff = (y.double() - ref.double()).abs()
+    ulp = bf16_ulp(ref)
+    assert torch.all(diff <= ulp + gamma * mag), float((diff - ulp - gamma * mag).max())
+    within_1ulp = float((diff <= ulp).double().mean())
+    assert within_1ulp > 0.999, within_1ulp
+    return within_1ulp
+
+
+@pytest.mark.parametrize("M", [1, 16])
+def test_w8a16_decode(M):
+    d = workload(4, M)
+    _check_w8a16(d["x"], d["q_w"], d["s_ch"])
+
+
+def test_w8a16_prefill_sampled_rows():
+    d = workload(4, 8192)
+    rows = [0, 1, 511, 512, 513, 4095, 8191]
+    _check_w8a16(d["x"], d["q_w"], d["s_ch"], rows=rows)
+
+
+@pytest.mark.parametrize("M,N,K", [(3, 144, 256), (33, 256, 640)])
+def test_w8a16_shapes(M, N, K):
+    x = inputs.gen_x(M, K, 5)
+    q_w = torch.randint(-127, 128, (N, K), dtype=torch.int8)
+    s_ch = torch.rand(N) * 1e-3 + 1e-5
+    _check_w8a16(x, q_w, s_ch)
+
+
+# ----------------------------------------------------------- error codes
+
+def test_error_codes():
+    q = torch.zeros((8, 256), dtype=torch.int8, device="cuda")
+    w = torch.zeros((32, 256), dtype=torch.int8, device="cuda")
+    s8 = torch.ones(8, device="cuda")
+    s32 = torch.ones(32, device="cuda")
+    with pytest.raises(sq.SqError) as e:
+        sq.w8a8_scaled_mm(q[:, :200].contiguous(), s8, w[:, :200].contiguous(), s32)
+    assert e.value.code == 2
+    wb = torch.zeros((24, 256), dtype=torch.int8, device="cuda")
+    with pytest.raises(sq.SqError) as e:
+        sq.w8a8_scaled_mm(q, s8, wb, torch.ones(24, device="cuda"))
+    assert e.value.code == 2
+    L = sq.lib()
+    y = torch.empty((8, 32), dtype=torch.bfloat16, device="cuda")
+    import ctypes
+    rc = L.w8a8_scaled_mm(ctypes.c_void_p(q.data_ptr() + 1), ctypes.c_void_p(s8.data_ptr()),
+                          ctypes.c_void_p(w.data_ptr()), ctypes.c_void_p(s32.data_ptr()),
+                          ctypes.c_void_p(y.data_ptr()), 8, 32, 256, None, 0, None)
+    assert rc == 3
+    rc = L.w8a8_scaled_mm(None, ctypes.c_void_p(s8.data_ptr()), ctypes.c_void_p(w.data_ptr()),
+                          ctypes.c_void_p(s32.data_ptr()), ctypes.c_void_p(y.data_ptr()),
+                          8, 32, 256, None, 0, None)
+    assert rc == 1
+    # small M needs workspace: none given
+    rc = L.w8a8_scaled_mm(ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(s8.data_ptr()),
+                          ctypes.c_void_p(w.data_ptr()), ctypes.c_void_p(s32.data_ptr()),
+                          ctypes.c_void_p(y.data_ptr()), 8, 32, 256, None, 0, None)
+    assert rc == 4
+    # M = 0 is a no-op
+    assert L.w8a8_scaled_mm(None, None, None, None, None, 0, 32, 256, None, 0, None) == 0
+    sq.check_device_error()

@@ -1,0 +1,206 @@
+"""Python binding of libsqint8.so (the B200 SmoothQuant W8A8 INT8 linear layer).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI of include/sqint8.h.  PyTorch supplies device
+memory and the current stream.  There is no CPU fallback: if the library
+cannot be loaded, every call raises.
+
+Functions (CUDA tensors in, CUDA tensors out, on the current stream):
+  quant_per_token(x, inv_s)            -> (q_a int8 [M,K], s_tok f32 [M])
+  w8a8_scaled_mm(q_a, s_tok, q_w, s_ch) -> y bf16 [M,N]
+  w8a8_gs128_mm(q_a, s_tok, q_w, s_blk) -> y bf16 [M,N]
+  w8a16_mm(x, q_w, s_ch)               -> y bf16 [M,N]
+  w8a8_mm_i32(q_a, q_w)                -> acc int32 [M,N]
+  linear_w8a8(x, inv_s, q_w, s_ch)     -> y bf16 [M,N] (quant + GEMM)
+  smooth_factors(x, w, cap, floor)     -> (s f32 [K], inv_s f32 [K])
+  quant_weight(w, smooth, group)       -> (q_w int8 [N,K], scales)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsqint8.so")
+
+OP_W8A8, OP_GS128, OP_W8A16, OP_W8A8_I32 = 0, 1, 2, 3
+_STATUS = {0: "ok", 1: "null pointer", 2: "unsupported shape", 3: "pointer not 16-byte aligned",
+           4: "workspace missing or too small", 5: "CUDA error", 6: "kernel wait timed out"}
+
+
+class SqError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn}: {_STATUS.get(code, 'unknown status')} (sq_status {code})")
+        self.code = code
+
+
+_lib = None
+_lock = threading.Lock()
+
+
+def lib() -> ctypes.CDLL:
+    """Load libsqint8.so (built by build.py); raises if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                                   "`python -m w8a8_int8_quantized_sq_b200.build`")
+            L = ctypes.CDLL(LIB_PATH)
+            vp, i64, sz, dbl = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_double
+            sig = {
+                "sq_quant_per_token": [vp, vp, vp, vp, i64, i64, vp],
+                "w8a8_scaled_mm": [vp, vp, vp, vp, vp, i64, i64, i64, vp, sz, vp],
+                "w8a8_gs128_mm": [vp, vp, vp, vp, vp, i64, i64, i64, vp, sz, vp],
+                "w8a16_mm": [vp, vp, vp, vp, i64, i64, i64, vp, sz, vp],
+                "w8a8_mm_i32": [vp, vp, vp, i64, i64, i64, vp, sz, vp],
+                "sq_smooth_factors": [vp, i64, vp, i64, i64, dbl, dbl, vp, vp, vp],
+                "sq_quant_weight": [vp, vp, vp, vp, i64, i64, i64, vp],
+                "sq_check_device_error": [ctypes.c_int],
+            }
+            for name, args in sig.items():
+                f = getattr(L, name)
+                f.argtypes = args
+                f.restype = ctypes.c_int
+            L.sq_workspace_bytes.argtypes = [ctypes.c_int, i64, i64, i64]
+            L.sq_workspace_bytes.restype = ctypes.c_size_t
+            L.sq_status_string.argtypes = [ctypes.c_int]
+            L.sq_status_string.restype = ctypes.c_char_p
+            _lib = L
+    return _lib
+
+
+EXPORTS = ("sq_quant_per_token", "w8a8_scaled_mm", "w8a8_gs128_mm", "w8a16_mm",
+           "sq_workspace_bytes", "w8a8_mm_i32", "sq_smooth_factors", "sq_quant_weight",
+           "sq_check_device_error", "sq_status_string")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _check(fn: str, rc: int) -> None:
+    if rc != 0:
+        raise SqError(fn, rc)
+
+
+# One zero-initialised workspace per (device, stream).  The kernels leave
+# their counters at zero, so it is reused without clearing; calls sharing a
+# stream are ordered, calls on different streams get different workspaces.
+_ws = {}
+
+
+def workspace(op: int, M: int, N: int, K: int, device) -> Tuple[Optional[torch.Tensor], int]:
+    need = lib().sq_workspace_bytes(op, M, N, K)
+    if need == 0:
+        return None, 0
+    dev = torch.device(device)
+    key = (dev.index, torch.cuda.current_stream(dev).cuda_stream)
+    buf = _ws.get(key)
+    if buf is None or buf.numel() < need:
+        buf = torch.zeros(max(need, 1 << 20), dtype=torch.uint8, device=dev)
+        _ws[key] = buf
+    return buf, buf.numel()
+
+
+def reset_workspaces() -> None:
+    """Drop cached workspaces (e.g. after a kernel reported a timeout)."""
+    _ws.clear()
+
+
+def quant_per_token(x: torch.Tensor, inv_s: Optional[torch.Tensor] = None):
+    assert x.dtype == torch.bfloat16 and x.dim() == 2
+    M, K = x.shape
+    q = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    s = torch.empty((M,), dtype=torch.float32, device=x.device)
+    _check("sq_quant_per_token", lib().sq_quant_per_token(
+        _ptr(x), _ptr(inv_s), _ptr(q), _ptr(s), M, K, _stream(x.device)))
+    return q, s
+
+
+def w8a8_scaled_mm(q_a, s_tok, q_w, s_ch, out: Optional[torch.Tensor] = None):
+    M, K = q_a.shape
+    N = q_w.shape[0]
+    y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=q_a.device)
+    ws, wsb = workspace(OP_W8A8, M, N, K, q_a.device)
+    _check("w8a8_scaled_mm", lib().w8a8_scaled_mm(
+        _ptr(q_a), _ptr(s_tok), _ptr(q_w), _ptr(s_ch), _ptr(y), M, N, K, _ptr(ws), wsb,
+        _stream(q_a.device)))
+    return y
+
+
+def w8a8_mm_i32(q_a, q_w):
+    M, K = q_a.shape
+    N = q_w.shape[0]
+    acc = torch.empty((M, N), dtype=torch.int32, device=q_a.device)
+    ws, wsb = workspace(OP_W8A8_I32, M, N, K, q_a.device)
+    _check("w8a8_mm_i32", lib().w8a8_mm_i32(
+        _ptr(q_a), _ptr(q_w), _ptr(acc), M, N, K, _ptr(ws), wsb, _stream(q_a.device)))
+    return acc
+
+
+def w8a8_gs128_mm(q_a, s_tok, q_w, s_blk):
+    M, K = q_a.shape
+    N = q_w.shape[0]
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=q_a.device)
+    ws, wsb = workspace(OP_GS128, M, N, K, q_a.device)
+    _check("w8a8_gs128_mm", lib().w8a8_gs128_mm(
+        _ptr(q_a), _ptr(s_tok), _ptr(q_w), _ptr(s_blk), _ptr(y), M, N, K, _ptr(ws), wsb,
+        _stream(q_a.device)))
+    return y
+
+
+def w8a16_mm(x, q_w, s_ch):
+    M, K = x.shape
+    N = q_w.shape[0]
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    ws, wsb = workspace(OP_W8A16, M, N, K, x.device)
+    _check("w8a16_mm", lib().w8a16_mm(
+        _ptr(x), _ptr(q_w), _ptr(s_ch), _ptr(y), M, N, K, _ptr(ws), wsb, _stream(x.device)))
+    return y
+
+
+def linear_w8a8(x, inv_s, q_w, s_ch):
+    """y = W8A8 linear layer: per-token quant with the 1/s fold, then the GEMM."""
+    q_a, s_tok = quant_per_token(x, inv_s)
+    return w8a8_scaled_mm(q_a, s_tok, q_w, s_ch)
+
+
+def smooth_factors(x, w, cap: float = 16.0, floor: float = 1e-5):
+    M, K = x.shape
+    N = w.shape[0]
+    s = torch.empty((K,), dtype=torch.float32, device=x.device)
+    inv = torch.empty((K,), dtype=torch.float32, device=x.device)
+    _check("sq_smooth_factors", lib().sq_smooth_factors(
+        _ptr(x), M, _ptr(w), N, K, cap, floor, _ptr(s), _ptr(inv), _stream(x.device)))
+    return s, inv
+
+
+def quant_weight(w, smooth: Optional[torch.Tensor] = None, group: int = 0):
+    N, K = w.shape
+    q = torch.empty((N, K), dtype=torch.int8, device=w.device)
+    sc = torch.empty((N, K // group) if group else (N,), dtype=torch.float32, device=w.device)
+    _check("sq_quant_weight", lib().sq_quant_weight(
+        _ptr(w), _ptr(smooth), _ptr(q), _ptr(sc), N, K, group, _stream(w.device)))
+    return q, sc
+
+
+def check_device_error(reset: bool = True) -> None:
+    """Synchronise; raise SqError if a kernel latched a wait timeout."""
+    _check("sq_check_device_error", lib().sq_check_device_error(1 if reset else 0))

@@ -1,0 +1,529 @@
+// gemm.cuh -- persistent, warp-specialised tcgen05 GEMM for sm_100a.
+//
+//   warp 0      : TMA producer (one elected thread) filling a ring of
+//                 shared-memory stages, each one 128-byte-wide K block of
+//                 A (128 rows) and B (BN rows), 128-byte swizzled.
+//   warp 1      : allocates tensor memory; one thread issues tcgen05.mma
+//                 (kind::i8 with int32 accumulators, or kind::f16 with BF16
+//                 operands and fp32 accumulators) into TMEM.
+//   warps 2..   : epilogue; tcgen05.ld of the accumulators, scale, convert,
+//                 store.  Double-buffered accumulators let the epilogue of
+//                 one tile overlap the mainloop of the next.
+//
+// "Rows" are the MMA M dimension (operand A) and "columns" the MMA N
+// dimension (operand B).  With SWAP = false A holds the tokens and B the
+// output channels; with SWAP = true (small token counts) A holds the weight
+// rows and B the tokens, so that the 128-row MMA tile is filled by weights.
+//
+// Schedules: tile-strided (CTA b takes tiles b, b+G, ...) or stream-K (CTA b
+// takes the contiguous range [b*T/G, (b+1)*T/G) of the T = tiles x K-blocks
+// iterations).  A tile split across CTAs is combined by the last CTA to
+// finish its part: every part is written to a per-CTA slot of the
+// workspace, an atomic counter per tile elects the last arrival, which sums
+// the parts in CTA order and runs the epilogue, then resets the counter.
+//
+// EPI_GS128 (group-size-128 weight scales): every 128-wide K block is MMA'd
+// into its own TMEM buffer that starts at the int32 pattern of 1.5 * 2^23,
+// so the block partial P arrives as the float 1.5 * 2^23 + P exactly and one
+// subtraction recovers f32(P); the epilogue warps then accumulate
+// fmaf(f32(P), s_blk[n, kb], acc) in registers in K-block order and restore
+// the buffer's starting pattern for its next use.
+#pragma once
+#include "ptx.cuh"
+
+namespace sq {
+
+enum : int { EPI_SCALE = 0, EPI_I32 = 1, EPI_GS128 = 2 };
+
+struct GemmArgs {
+  int R, C;               // MMA rows (A rows) and columns (B rows)
+  int kb_total;           // K blocks of 128 bytes
+  int tiles_r, tiles_c, num_tiles;
+  int stream_k;           // 0: tile-strided, 1: stream-K ranges
+  long long total_iters;  // num_tiles * kb_total
+  int M, N;               // output y is [M, N] row-major
+  const float* s_tok;     // [M] per-token scales (may be null: W8A16)
+  const float* s_ch;      // [N] per-channel scales
+  const float* s_blk;     // [N, kb_total] block scales (EPI_GS128)
+  void* out;              // bf16 [M, N] or int32 [M, N]
+  uint32_t* ws;           // stream-K slots [grid][2][128][BN] 32-bit words
+  unsigned int* ws_cnt;   // stream-K arrival counters [num_tiles]
+};
+
+__host__ __device__ constexpr int pow2_at_least(int v) {
+  int p = 32;
+  while (p < v) p <<= 1;
+  return p;
+}
+
+template <bool I8_, int BN_, int STAGES_, bool SWAP_, int EPI_>
+struct GemmCfg {
+  static constexpr bool I8 = I8_;
+  static constexpr int BN = BN_;
+  static constexpr int STAGES = STAGES_;
+  static constexpr bool SWAP = SWAP_;
+  static constexpr int EPI = EPI_;
+  static constexpr int BM = 128;
+  static constexpr int KB_BYTES = 128;
+  static constexpr int KB_ELEMS = I8 ? 128 : 64;
+  static constexpr int A_BYTES = BM * KB_BYTES;
+  static constexpr int B_BYTES = BN * KB_BYTES;
+  static constexpr int NE = (EPI == EPI_GS128) ? 8 : 4;  // epilogue warps
+  static constexpr int THREADS = 64 + NE * 32;
+  static constexpr int NACC = (EPI == EPI_GS128) ? 4 : 2;
+  static constexpr int TMEM_COLS = pow2_at_least(NACC * BN);
+  static constexpr int CW = BN < 32 ? BN : 32;  // columns per tcgen05.ld
+  static constexpr int CPT = BN / (NE / 4);     // columns owned by one epilogue thread
+  static constexpr int SBLK_STRIDE = BN + 4;    // floats per K block in the staged s_blk
+  // shared memory carve-up (offsets from a 1024-byte aligned base)
+  static constexpr int OFF_A = 0;
+  static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
+  static constexpr int OFF_BAR = OFF_B + STAGES * B_BYTES;
+  static constexpr int NUM_BARS = 2 * STAGES + 2 * NACC + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  static constexpr int OFF_SBLK = (OFF_MISC + 16 + 15) / 16 * 16;
+  static constexpr int smem_bytes(int kb_total) {
+    return 1024 + OFF_SBLK + (EPI == EPI_GS128 ? kb_total * SBLK_STRIDE * 4 : 0);
+  }
+  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N for M = 128");
+  static_assert(EPI != EPI_GS128 || (I8 && !SWAP && BN % 64 == 0), "gs128 layout");
+  static_assert(TMEM_COLS <= 512, "tensor memory");
+};
+
+struct Seg {
+  int tile, kb0, kb1;
+};
+
+__device__ __forceinline__ long long sk_start(long long b, long long G, long long T) {
+  return b * T / G;
+}
+// CTA whose stream-K range contains iteration i.
+__device__ __forceinline__ long long sk_owner(long long i, long long G, long long T) {
+  return ((i + 1) * G + T - 1) / T - 1;
+}
+
+struct SegIter {
+  long long pos, end;
+  __device__ __forceinline__ void init(const GemmArgs& g) {
+    if (g.stream_k) {
+      pos = sk_start(blockIdx.x, gridDim.x, g.total_iters);
+      end = sk_start(blockIdx.x + 1, gridDim.x, g.total_iters);
+    } else {
+      pos = blockIdx.x;
+      end = g.num_tiles;
+    }
+  }
+  __device__ __forceinline__ bool next(const GemmArgs& g, Seg& s) {
+    if (pos >= end) return false;
+    if (g.stream_k) {
+      s.tile = static_cast<int>(pos / g.kb_total);
+      s.kb0 = static_cast<int>(pos % g.kb_total);
+      const long long rem = end - pos;
+      s.kb1 = static_cast<int>(rem < g.kb_total - s.kb0 ? s.kb0 + rem : g.kb_total);
+      pos += s.kb1 - s.kb0;
+    } else {
+      s.tile = static_cast<int>(pos);
+      s.kb0 = 0;
+      s.kb1 = g.kb_total;
+      pos += gridDim.x;
+    }
+    return true;
+  }
+};
+
+// --------------------------------------------------------------- epilogue
+// Scale/convert/store CW accumulator columns [c0, c0 + CW) of MMA row rr of
+// tile (rt, ct).  v holds int32 (I8) or fp32 bits (BF16) accumulators.
+template <class Cfg>
+__device__ __forceinline__ void store_chunk(const GemmArgs& g, int rt, int ct, int rr, int c0,
+                                            const uint32_t (&v)[Cfg::CW]) {
+  constexpr int CW = Cfg::CW;
+  const int r = rt * Cfg::BM + rr;
+  const int cb = ct * Cfg::BN + c0;
+  if constexpr (!Cfg::SWAP) {
+    const int m = r;
+    if (m >= g.M) return;
+    if constexpr (Cfg::EPI == EPI_I32) {
+      int32_t* out = static_cast<int32_t*>(g.out) + static_cast<size_t>(m) * g.N;
+#pragma unroll
+      for (int j = 0; j < CW; j += 4) {
+        const int n = cb + j;
+        if (n + 4 <= g.N)
+          *reinterpret_cast<int4*>(out + n) = make_int4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+      }
+    } else {
+      __nv_bfloat16* out = static_cast<__nv_bfloat16*>(g.out) + static_cast<size_t>(m) * g.N;
+      const float st = (Cfg::I8 && g.s_tok) ? __ldg(g.s_tok + m) : 1.0f;
+#pragma unroll
+      for (int j = 0; j < CW; j += 8) {
+        const int n = cb + j;
+        if (n + 8 > g.N) break;
+        const float4 c0v = __ldg(reinterpret_cast<const float4*>(g.s_ch + n));
+        const float4 c1v = __ldg(reinterpret_cast<const float4*>(g.s_ch + n) + 1);
+        const float sc[8] = {c0v.x, c0v.y, c0v.z, c0v.w, c1v.x, c1v.y, c1v.z, c1v.w};
+        float f[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          if constexpr (Cfg::I8) {
+            f[i] = __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(v[j + i])), st), sc[i]);
+          } else {
+            f[i] = __fmul_rn(__uint_as_float(v[j + i]), sc[i]);
+          }
+        }
+        *reinterpret_cast<uint4*>(out + n) =
+            make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                       pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+      }
+    }
+  } else {
+    const int n = r;
+    if (n >= g.N) return;
+    if constexpr (Cfg::EPI == EPI_I32) {
+      int32_t* out = static_cast<int32_t*>(g.out);
+#pragma unroll
+      for (int j = 0; j < CW; ++j) {
+        const int m = cb + j;
+        if (m < g.M) out[static_cast<size_t>(m) * g.N + n] = static_cast<int32_t>(v[j]);
+      }
+    } else {
+      __nv_bfloat16* out = static_cast<__nv_bfloat16*>(g.out);
+      const float sc = __ldg(g.s_ch + n);
+#pragma unroll
+      for (int j = 0; j < CW; ++j) {
+        const int m = cb + j;
+        if (m < g.M) {
+          float f;
+          if constexpr (Cfg::I8) {
+            const float st = g.s_tok ? __ldg(g.s_tok + m) : 1.0f;
+            f = __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(v[j])), st), sc);
+          } else {
+            f = __fmul_rn(__uint_as_float(v[j]), sc);
+          }
+          out[static_cast<size_t>(m) * g.N + n] = __float2bfloat16_rn(f);
+        }
+      }
+    }
+  }
+}
+
+template <class Cfg>
+__device__ __forceinline__ void tmem_ld_chunk(uint32_t taddr, uint32_t (&v)[Cfg::CW]) {
+  if constexpr (Cfg::CW == 32) tmem_ld32(taddr, v);
+  else tmem_ld16(taddr, v);
+}
+
+// ------------------------------------------------------------------ kernel
+template <class Cfg>
+__global__ void __launch_bounds__(Cfg::THREADS, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const GemmArgs g) {
+  constexpr int BN = Cfg::BN, STAGES = Cfg::STAGES, NACC = Cfg::NACC, NE = Cfg::NE;
+  constexpr int CW = Cfg::CW;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* smA = smem + Cfg::OFF_A;
+  uint8_t* smB = smem + Cfg::OFF_B;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + STAGES;
+  uint64_t* tfull = bars + 2 * STAGES;
+  uint64_t* tempty = tfull + NACC;
+  uint64_t* drain = tempty + NACC;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::OFF_MISC + 4);
+  volatile int* sk_flag = reinterpret_cast<volatile int*>(smem + Cfg::OFF_MISC + 8);
+  float* sblk = reinterpret_cast<float*>(smem + Cfg::OFF_SBLK);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, 1);
+    }
+    for (int a = 0; a < NACC; ++a) {
+      mbar_init(tfull + a, 1);
+      mbar_init(tempty + a, NE);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    *sk_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, Cfg::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmA);
+      tma_prefetch_desc(&tmB);
+      uint32_t stage = 0, phase = 0;
+      long long fills = 0;
+      SegIter it;
+      it.init(g);
+      Seg s;
+      bool ok = true;
+      while (ok && it.next(g, s)) {
+        const int rt = s.tile % g.tiles_r, ct = s.tile / g.tiles_r;
+        for (int kb = s.kb0; kb < s.kb1; ++kb) {
+          if (!wait_bounded(empty + stage, phase ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(full + stage, Cfg::A_BYTES + Cfg::B_BYTES);
+          tma_load_2d(smA + stage * Cfg::A_BYTES, &tmA, kb * Cfg::KB_ELEMS, rt * Cfg::BM,
+                      full + stage);
+          tma_load_2d(smB + stage * Cfg::B_BYTES, &tmB, kb * Cfg::KB_ELEMS, ct * BN, full + stage);
+          ++fills;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // no copy may still be writing shared memory when the CTA exits
+      for (int st = 0; st < STAGES; ++st) {
+        const long long n = fills / STAGES + (st < fills % STAGES ? 1 : 0);
+        if (n > 0) wait_drain(full + st, static_cast<uint32_t>((n - 1) & 1));
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = Cfg::I8 ? idesc_i8_s32(BN) : idesc_bf16_f32(BN);
+      uint32_t stage = 0, phase = 0;
+      uint32_t local = 0;
+      SegIter it;
+      it.init(g);
+      Seg s;
+      bool ok = true;
+      while (ok && it.next(g, s)) {
+        if constexpr (Cfg::EPI == EPI_GS128) {
+          for (int kb = s.kb0; kb < s.kb1 && ok; ++kb, ++local) {
+            const uint32_t p = local % NACC, u = local / NACC;
+            if (!wait_bounded(tempty + p, u & 1u, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            if (!wait_bounded(full + stage, phase, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t sa = smem_u32(smA + stage * Cfg::A_BYTES);
+            const uint32_t sb = smem_u32(smB + stage * Cfg::B_BYTES);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              mma_i8(tmem + p * BN, smem_desc_sw128(sa + k * 32), smem_desc_sw128(sb + k * 32),
+                     idesc, 1u);
+            mma_commit(empty + stage);
+            mma_commit(tfull + p);
+            if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          }
+        } else {
+          const uint32_t a = local % NACC, u = local / NACC;
+          if (!wait_bounded(tempty + a, (u & 1u) ^ 1u, abort_flag)) break;
+          tc_fence_after();
+          const uint32_t d = tmem + a * BN;
+          for (int kb = s.kb0; kb < s.kb1; ++kb) {
+            if (!wait_bounded(full + stage, phase, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t sa = smem_u32(smA + stage * Cfg::A_BYTES);
+            const uint32_t sb = smem_u32(smB + stage * Cfg::B_BYTES);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const uint32_t accum = (kb > s.kb0 || k > 0) ? 1u : 0u;
+              if constexpr (Cfg::I8)
+                mma_i8(d, smem_desc_sw128(sa + k * 32), smem_desc_sw128(sb + k * 32), idesc, accum);
+              else
+                mma_bf16(d, smem_desc_sw128(sa + k * 32), smem_desc_sw128(sb + k * 32), idesc,
+                         accum);
+            }
+            mma_commit(empty + stage);
+            if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          }
+          if (!ok) break;
+          mma_commit(tfull + a);
+          ++local;
+        }
+      }
+      // every MMA issued by this thread has finished before TMEM is freed
+      mma_commit(drain);
+      wait_drain(drain, 0);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int ew = warp - 2;
+    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    const int rr = q * 32 + lane;
+    const int nthr = NE * 32;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16);
+    SegIter it;
+    it.init(g);
+    Seg s;
+    if constexpr (Cfg::EPI == EPI_GS128) {
+      constexpr int CPT = Cfg::CPT;
+      const int h = ew / 4;
+      const int col0 = h * CPT;
+      const int et = ew * 32 + lane;
+      // every buffer starts at the bias pattern; releasing it completes phase 0
+#pragma unroll
+      for (int p = 0; p < NACC; ++p)
+#pragma unroll
+        for (int c = 0; c < CPT; c += 32) tmem_st32_const(lane_base + p * BN + col0 + c, 0x4B400000u);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0)
+        for (int p = 0; p < NACC; ++p) mbar_arrive(tempty + p);
+      uint32_t local = 0;
+      bool ok = true;
+      while (ok && it.next(g, s)) {
+        const int rt = s.tile % g.tiles_r, ct = s.tile / g.tiles_r;
+        // stage this tile's block scales, transposed to [kb][n]
+        named_bar_sync(1, nthr);
+        const int total = g.kb_total * BN;
+        for (int idx = et; idx < total; idx += nthr) {
+          const int j = idx / g.kb_total, kb = idx - j * g.kb_total;
+          const int n = ct * BN + j;
+          sblk[kb * Cfg::SBLK_STRIDE + j] = n < g.N ? __ldg(g.s_blk + static_cast<size_t>(n) * g.kb_total + kb) : 0.0f;
+        }
+        named_bar_sync(1, nthr);
+        float acc[CPT];
+#pragma unroll
+        for (int j = 0; j < CPT; ++j) acc[j] = 0.0f;
+        for (int kb = s.kb0; kb < s.kb1; ++kb, ++local) {
+          const uint32_t p = local % NACC, u = local / NACC;
+          const bool w_ok = wait_bounded(tfull + p, u & 1u, abort_flag);
+          if (named_bar_or(1, nthr, !w_ok)) { ok = false; break; }
+          tc_fence_after();
+          const float* sk = sblk + kb * Cfg::SBLK_STRIDE + col0;
+#pragma unroll
+          for (int c = 0; c < CPT; c += 32) {
+            uint32_t v[32];
+            const uint32_t ta = lane_base + p * BN + col0 + c;
+            tmem_ld32(ta, v);
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+              const float4 s4 = *reinterpret_cast<const float4*>(sk + c + j);
+              acc[c + j] = __fmaf_rn(__fsub_rn(__uint_as_float(v[j]), 12582912.0f), s4.x, acc[c + j]);
+              acc[c + j + 1] = __fmaf_rn(__fsub_rn(__uint_as_float(v[j + 1]), 12582912.0f), s4.y, acc[c + j + 1]);
+              acc[c + j + 2] = __fmaf_rn(__fsub_rn(__uint_as_float(v[j + 2]), 12582912.0f), s4.z, acc[c + j + 2]);
+              acc[c + j + 3] = __fmaf_rn(__fsub_rn(__uint_as_float(v[j + 3]), 12582912.0f), s4.w, acc[c + j + 3]);
+            }
+            tmem_st32_const(ta, 0x4B400000u);
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(tempty + p);
+        }
+        if (!ok) break;
+        const int m = rt * Cfg::BM + rr;
+        if (m < g.M) {
+          const float st = __ldg(g.s_tok + m);
+          __nv_bfloat16* out = static_cast<__nv_bfloat16*>(g.out) + static_cast<size_t>(m) * g.N;
+#pragma unroll
+          for (int j = 0; j < CPT; j += 8) {
+            const int n = ct * BN + col0 + j;
+            if (n + 8 <= g.N)
+              *reinterpret_cast<uint4*>(out + n) = make_uint4(
+                  pack_bf16x2(__fmul_rn(acc[j], st), __fmul_rn(acc[j + 1], st)),
+                  pack_bf16x2(__fmul_rn(acc[j + 2], st), __fmul_rn(acc[j + 3], st)),
+                  pack_bf16x2(__fmul_rn(acc[j + 4], st), __fmul_rn(acc[j + 5], st)),
+                  pack_bf16x2(__fmul_rn(acc[j + 6], st), __fmul_rn(acc[j + 7], st)));
+          }
+        }
+      }
+    } else {
+      uint32_t local = 0;
+      const long long G = gridDim.x, T = g.total_iters;
+      while (it.next(g, s)) {
+        const uint32_t a = local % NACC, u = local / NACC;
+        const bool w_ok = wait_bounded(tfull + a, u & 1u, abort_flag);
+        if (named_bar_or(1, nthr, !w_ok)) break;
+        tc_fence_after();
+        const int rt = s.tile % g.tiles_r, ct = s.tile / g.tiles_r;
+        const uint32_t tb = lane_base + a * BN;
+        if (s.kb0 == 0 && s.kb1 == g.kb_total) {
+#pragma unroll 1
+          for (int c = 0; c < BN; c += CW) {
+            uint32_t v[CW];
+            tmem_ld_chunk<Cfg>(tb + c, v);
+            store_chunk<Cfg>(g, rt, ct, rr, c, v);
+          }
+        } else {
+          // stream-K part of a tile: publish, count, and the last arrival reduces
+          const long long it0 = static_cast<long long>(s.tile) * g.kb_total;
+          const long long b_lo = sk_owner(it0, G, T);
+          const long long b_hi = sk_owner(it0 + g.kb_total - 1, G, T);
+          const int slot = sk_start(blockIdx.x, G, T) >= it0 ? 0 : 1;
+          uint32_t* wrow = g.ws + (static_cast<size_t>(blockIdx.x * 2 + slot) * Cfg::BM + rr) * BN;
+#pragma unroll 1
+          for (int c = 0; c < BN; c += CW) {
+            uint32_t v[CW];
+            tmem_ld_chunk<Cfg>(tb + c, v);
+#pragma unroll
+            for (int j = 0; j < CW; j += 4)
+              *reinterpret_cast<uint4*>(wrow + c + j) = make_uint4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+          }
+          __threadfence();
+          named_bar_sync(1, nthr);
+          if (ew == 0 && lane == 0) {
+            const unsigned prev = atomicAdd(g.ws_cnt + s.tile, 1u);
+            const int last = prev == static_cast<unsigned>(b_hi - b_lo);
+            if (last) atomicExch(g.ws_cnt + s.tile, 0u);
+            *sk_flag = last;
+          }
+          named_bar_sync(1, nthr);
+          if (*sk_flag) {
+            __threadfence();
+#pragma unroll 1
+            for (int c = 0; c < BN; c += CW) {
+              uint32_t v[CW];
+#pragma unroll
+              for (int j = 0; j < CW; ++j) v[j] = 0u;
+              for (long long b = b_lo; b <= b_hi; ++b) {
+                const int sl = sk_start(b, G, T) >= it0 ? 0 : 1;
+                const uint32_t* prow =
+                    g.ws + (static_cast<size_t>(b * 2 + sl) * Cfg::BM + rr) * BN + c;
+#pragma unroll
+                for (int j = 0; j < CW; j += 4) {
+                  const int4 w = ld_cg_v4(prow + j);
+                  const uint32_t wv[4] = {static_cast<uint32_t>(w.x), static_cast<uint32_t>(w.y),
+                                          static_cast<uint32_t>(w.z), static_cast<uint32_t>(w.w)};
+#pragma unroll
+                  for (int i = 0; i < 4; ++i) {
+                    if constexpr (Cfg::I8)
+                      v[j + i] = static_cast<uint32_t>(static_cast<int32_t>(v[j + i]) +
+                                                       static_cast<int32_t>(wv[i]));
+                    else
+                      v[j + i] = __float_as_uint(__fadd_rn(__uint_as_float(v[j + i]),
+                                                           __uint_as_float(wv[i])));
+                  }
+                }
+              }
+              store_chunk<Cfg>(g, rt, ct, rr, c, v);
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tempty + a);
+        ++local;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, Cfg::TMEM_COLS);
+  }
+}
+
+}  // namespace sq

@@ -1,0 +1,394 @@
+// sqint8.cu -- host side of the C ABI declared in include/sqint8.h:
+// argument checks, launch planning, tensor-map encoding and kernel launches.
+// The library holds no device memory of its own except one error word.
+#include <atomic>
+#include <mutex>
+
+#include "../../include/sqint8.h"
+#include "gemm.cuh"
+#include "quant.cuh"
+
+using namespace sq;
+
+namespace {
+
+constexpr int64_t kMaxK = 131072;  // K * 127 * 127 < 2^31
+// Every workspace starts with this many bytes of stream-K arrival counters
+// (one 32-bit word per tile).  Nothing else is ever written there, so the
+// region stays zero across calls of different operations and sizes that
+// share one workspace.  Split-K scratch and converted weights follow it.
+constexpr size_t kCounterBytes = 65536;
+constexpr int64_t kMaxCounterTiles = static_cast<int64_t>(kCounterBytes / 4);
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// K-major 2-D operand: rows of `inner` elements, box of box_inner x box_rows,
+// 128-byte swizzle, out-of-bounds rows read as zero.
+bool make_map(CUtensorMap* m, const void* ptr, bool bf16, uint64_t inner, uint64_t rows,
+              uint32_t box_inner, uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const uint64_t esz = bf16 ? 2 : 1;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner * esz};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+                   const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int num_sms() {
+  static std::atomic<int> cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (dev < 0 || dev >= 64) return 0;
+  int v = cache[dev].load(std::memory_order_relaxed);
+  if (v > 0) return v;
+  if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  cache[dev].store(v, std::memory_order_relaxed);
+  return v;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
+
+sq_status check_mnk(int64_t M, int64_t N, int64_t K) {
+  if (M < 0 || N <= 0 || K <= 0) return SQ_ERR_SHAPE;
+  if (N % 16 || K % 128 || K > kMaxK) return SQ_ERR_SHAPE;
+  if (M > (1ll << 31) - 1 || N > (1ll << 31) - 1) return SQ_ERR_SHAPE;
+  return SQ_OK;
+}
+
+sq_status launch_status() {
+  return cudaGetLastError() == cudaSuccess ? SQ_OK : SQ_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------- planning
+enum GemmKind { GK_I8_SCALE = 0, GK_I8_I32 = 1, GK_GS128 = 2, GK_BF16 = 3 };
+
+struct GemmPlan {
+  bool swap;
+  int bn;
+  bool stream_k;
+  int grid;
+  int tiles_r, tiles_c;
+  int kb_total;
+  long long total_iters;
+  size_t ws_bytes;  // counter region + stream-K slots (0: no workspace)
+};
+
+GemmPlan plan_gemm(GemmKind kind, int64_t M, int64_t N, int64_t K, int sms) {
+  GemmPlan p{};
+  const bool i8 = kind != GK_BF16;
+  p.kb_total = static_cast<int>(K / (i8 ? 128 : 64));
+  if (kind != GK_GS128 && M <= 32) {
+    p.swap = true;
+    p.bn = M <= 16 ? 16 : 32;
+    p.tiles_r = static_cast<int>((N + 127) / 128);
+    p.tiles_c = 1;
+    p.stream_k = true;
+    p.total_iters = static_cast<long long>(p.tiles_r) * p.kb_total;
+    p.grid = static_cast<int>(p.total_iters < sms ? p.total_iters : sms);
+    p.ws_bytes = kCounterBytes + static_cast<size_t>(p.grid) * 2 * 128 * p.bn * 4;
+  } else {
+    p.swap = false;
+    p.bn = kind == GK_GS128 ? 128 : 256;
+    p.tiles_r = static_cast<int>((M + 127) / 128);
+    p.tiles_c = static_cast<int>((N + p.bn - 1) / p.bn);
+    p.stream_k = false;
+    const long long tiles = static_cast<long long>(p.tiles_r) * p.tiles_c;
+    p.total_iters = tiles * p.kb_total;
+    p.grid = static_cast<int>(tiles < sms ? tiles : sms);
+    p.ws_bytes = 0;
+  }
+  return p;
+}
+
+template <class Cfg>
+sq_status launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& g, int grid,
+                      cudaStream_t st) {
+  const int smem = Cfg::smem_bytes(g.kb_total);
+  if (smem > 232448) return SQ_ERR_SHAPE;
+  if (cudaFuncSetAttribute(gemm_kernel<Cfg>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+      cudaSuccess)
+    return SQ_ERR_CUDA;
+  gemm_kernel<Cfg><<<grid, Cfg::THREADS, smem, st>>>(a, b, g);
+  return launch_status();
+}
+
+// act: q_a int8 [M,K] or x bf16 [M,K]; wt: q_w int8 [N,K] or bf16 [N,K].
+sq_status run_gemm(GemmKind kind, const void* act, const void* wt, const float* s_tok,
+                   const float* s_ch, const float* s_blk, void* out, int64_t M, int64_t N,
+                   int64_t K, void* ws, size_t ws_bytes, cudaStream_t st) {
+  const int sms = num_sms();
+  if (sms <= 0) return SQ_ERR_CUDA;
+  const GemmPlan p = plan_gemm(kind, M, N, K, sms);
+  if (p.stream_k && static_cast<int64_t>(p.tiles_r) * p.tiles_c > kMaxCounterTiles)
+    return SQ_ERR_SHAPE;
+  if (p.ws_bytes > 0 && (!ws || ws_bytes < p.ws_bytes)) return SQ_ERR_WORKSPACE;
+  if (ws && !aligned16(ws)) return SQ_ERR_ALIGN;
+  const bool bf16 = kind == GK_BF16;
+  const uint32_t kbe = bf16 ? 64 : 128;
+  CUtensorMap ta, tb;
+  const void* a_ptr = p.swap ? wt : act;
+  const void* b_ptr = p.swap ? act : wt;
+  const uint64_t a_rows = static_cast<uint64_t>(p.swap ? N : M);
+  const uint64_t b_rows = static_cast<uint64_t>(p.swap ? M : N);
+  if (!make_map(&ta, a_ptr, bf16, static_cast<uint64_t>(K), a_rows, kbe, 128)) return SQ_ERR_CUDA;
+  if (!make_map(&tb, b_ptr, bf16, static_cast<uint64_t>(K), b_rows, kbe, p.bn)) return SQ_ERR_CUDA;
+
+  GemmArgs g{};
+  g.R = static_cast<int>(p.swap ? N : M);
+  g.C = static_cast<int>(p.swap ? M : N);
+  g.kb_total = p.kb_total;
+  g.tiles_r = p.tiles_r;
+  g.tiles_c = p.tiles_c;
+  g.num_tiles = p.tiles_r * p.tiles_c;
+  g.stream_k = p.stream_k ? 1 : 0;
+  g.total_iters = p.total_iters;
+  g.M = static_cast<int>(M);
+  g.N = static_cast<int>(N);
+  g.s_tok = s_tok;
+  g.s_ch = s_ch;
+  g.s_blk = s_blk;
+  g.out = out;
+  g.ws_cnt = p.ws_bytes ? static_cast<unsigned int*>(ws) : nullptr;
+  g.ws = p.ws_bytes ? reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + kCounterBytes)
+                    : nullptr;
+
+  switch (kind) {
+    case GK_I8_SCALE:
+      if (p.swap && p.bn == 16)
+        return launch_gemm<GemmCfg<true, 16, 8, true, EPI_SCALE>>(ta, tb, g, p.grid, st);
+      if (p.swap)
+        return launch_gemm<GemmCfg<true, 32, 8, true, EPI_SCALE>>(ta, tb, g, p.grid, st);
+      return launch_gemm<GemmCfg<true, 256, 4, false, EPI_SCALE>>(ta, tb, g, p.grid, st);
+    case GK_I8_I32:
+      if (p.swap && p.bn == 16)
+        return launch_gemm<GemmCfg<true, 16, 8, true, EPI_I32>>(ta, tb, g, p.grid, st);
+      if (p.swap)
+        return launch_gemm<GemmCfg<true, 32, 8, true, EPI_I32>>(ta, tb, g, p.grid, st);
+      return launch_gemm<GemmCfg<true, 256, 4, false, EPI_I32>>(ta, tb, g, p.grid, st);
+    case GK_GS128:
+      return launch_gemm<GemmCfg<true, 128, 4, false, EPI_GS128>>(ta, tb, g, p.grid, st);
+    case GK_BF16:
+      if (p.swap && p.bn == 16)
+        return launch_gemm<GemmCfg<false, 16, 8, true, EPI_SCALE>>(ta, tb, g, p.grid, st);
+      if (p.swap)
+        return launch_gemm<GemmCfg<false, 32, 8, true, EPI_SCALE>>(ta, tb, g, p.grid, st);
+      return launch_gemm<GemmCfg<false, 256, 4, false, EPI_SCALE>>(ta, tb, g, p.grid, st);
+  }
+  return SQ_ERR_SHAPE;
+}
+
+// W8A16 workspace: [counter region][stream-K slots][bf16 weights N x K]
+size_t w8a16_ws_bytes(int64_t M, int64_t N, int64_t K, int sms, size_t* w_off) {
+  const GemmPlan p = plan_gemm(GK_BF16, M, N, K, sms);
+  const size_t off = align256(p.ws_bytes > kCounterBytes ? p.ws_bytes : kCounterBytes);
+  if (w_off) *w_off = off;
+  return off + static_cast<size_t>(N) * static_cast<size_t>(K) * 2;
+}
+
+template <int TPR, bool HAS_VEC>
+sq_status launch_quant(const void* x, const float* vec, int8_t* q, float* scales, int64_t nseg,
+                       int64_t K, int64_t group, cudaStream_t st) {
+  constexpr int SEGS = 256 / TPR;
+  const int64_t blocks = (nseg + SEGS - 1) / SEGS;
+  if (blocks > 2147483647ll) return SQ_ERR_SHAPE;
+  quant_rows_kernel<TPR, HAS_VEC><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(x), vec, q, scales, nseg, static_cast<int>(K),
+      static_cast<int>(group));
+  return launch_status();
+}
+
+sq_status quant_rows(const void* x, const float* vec, int8_t* q, float* scales, int64_t nseg,
+                     int64_t K, int64_t group, cudaStream_t st) {
+  if (nseg == 0) return SQ_OK;
+  if (group == 128) {
+    return vec ? launch_quant<8, true>(x, vec, q, scales, nseg, K, group, st)
+               : launch_quant<8, false>(x, vec, q, scales, nseg, K, group, st);
+  }
+  if (nseg >= 2048) {
+    return vec ? launch_quant<32, true>(x, vec, q, scales, nseg, K, group, st)
+               : launch_quant<32, false>(x, vec, q, scales, nseg, K, group, st);
+  }
+  return vec ? launch_quant<256, true>(x, vec, q, scales, nseg, K, group, st)
+             : launch_quant<256, false>(x, vec, q, scales, nseg, K, group, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* sq_status_string(sq_status s) {
+  switch (s) {
+    case SQ_OK: return "ok";
+    case SQ_ERR_NULL: return "null pointer";
+    case SQ_ERR_SHAPE: return "unsupported shape";
+    case SQ_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case SQ_ERR_WORKSPACE: return "workspace missing or too small";
+    case SQ_ERR_CUDA: return "CUDA error";
+    case SQ_ERR_TIMEOUT: return "kernel wait timed out";
+  }
+  return "unknown status";
+}
+
+sq_status sq_quant_per_token(const void* x_bf16, const float* inv_smooth, int8_t* q_i8,
+                             float* s_tok, int64_t M, int64_t K, void* stream) {
+  if (M < 0 || K <= 0 || K % 128 || K > kMaxK) return SQ_ERR_SHAPE;
+  if (M == 0) return SQ_OK;
+  if (!x_bf16 || !q_i8 || !s_tok) return SQ_ERR_NULL;
+  if (!aligned16(x_bf16) || !aligned16(q_i8) || !aligned16(s_tok) ||
+      (inv_smooth && !aligned16(inv_smooth)))
+    return SQ_ERR_ALIGN;
+  return quant_rows(x_bf16, inv_smooth, q_i8, s_tok, M, K, K, static_cast<cudaStream_t>(stream));
+}
+
+sq_status sq_quant_weight(const void* w_bf16, const float* smooth, int8_t* q_w, float* scales,
+                          int64_t N, int64_t K, int64_t group, void* stream) {
+  if (N < 0 || K <= 0 || K % 128 || K > kMaxK || (group != 0 && group != 128))
+    return SQ_ERR_SHAPE;
+  if (N == 0) return SQ_OK;
+  if (!w_bf16 || !q_w || !scales) return SQ_ERR_NULL;
+  if (!aligned16(w_bf16) || !aligned16(q_w) || !aligned16(scales) || (smooth && !aligned16(smooth)))
+    return SQ_ERR_ALIGN;
+  const int64_t g = group ? group : K;
+  return quant_rows(w_bf16, smooth, q_w, scales, N * (K / g), K, g,
+                    static_cast<cudaStream_t>(stream));
+}
+
+sq_status sq_smooth_factors(const void* x_bf16, int64_t M, const void* w_bf16, int64_t N,
+                            int64_t K, double cap, double floor_, float* s_out,
+                            float* inv_s_out, void* stream) {
+  if (M <= 0 || N <= 0 || K <= 0 || K % 128 || K > kMaxK) return SQ_ERR_SHAPE;
+  if (!x_bf16 || !w_bf16 || !s_out || !inv_s_out) return SQ_ERR_NULL;
+  if (!aligned16(x_bf16) || !aligned16(w_bf16) || !aligned16(s_out) || !aligned16(inv_s_out))
+    return SQ_ERR_ALIGN;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(s_out, 0, K * 4, st) != cudaSuccess) return SQ_ERR_CUDA;
+  if (cudaMemsetAsync(inv_s_out, 0, K * 4, st) != cudaSuccess) return SQ_ERR_CUDA;
+  const int rpb = 64;
+  const unsigned gx = static_cast<unsigned>((K / 8 + 255) / 256);
+  dim3 gxm(gx, static_cast<unsigned>((M + rpb - 1) / rpb));
+  colmax_kernel<<<gxm, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x_bf16), M,
+                                     static_cast<int>(K), rpb,
+                                     reinterpret_cast<unsigned int*>(s_out));
+  dim3 gwn(gx, static_cast<unsigned>((N + rpb - 1) / rpb));
+  colmax_kernel<<<gwn, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(w_bf16), N,
+                                     static_cast<int>(K), rpb,
+                                     reinterpret_cast<unsigned int*>(inv_s_out));
+  smooth_finalize_kernel<<<static_cast<unsigned>((K + 255) / 256), 256, 0, st>>>(
+      s_out, inv_s_out, static_cast<int>(K), cap, floor_);
+  return launch_status();
+}
+
+size_t sq_workspace_bytes(int op, int64_t M, int64_t N, int64_t K) {
+  if (check_mnk(M, N, K) != SQ_OK) return 0;
+  const int sms = num_sms();
+  if (sms <= 0) return 0;
+  switch (op) {
+    case SQ_OP_W8A8: return plan_gemm(GK_I8_SCALE, M, N, K, sms).ws_bytes;
+    case SQ_OP_W8A8_I32: return plan_gemm(GK_I8_I32, M, N, K, sms).ws_bytes;
+    case SQ_OP_GS128: return plan_gemm(GK_GS128, M, N, K, sms).ws_bytes;
+    case SQ_OP_W8A16: return w8a16_ws_bytes(M, N, K, sms, nullptr);
+  }
+  return 0;
+}
+
+sq_status w8a8_scaled_mm(const int8_t* q_a, const float* s_tok, const int8_t* q_w,
+                         const float* s_ch, void* y_bf16, int64_t M, int64_t N, int64_t K,
+                         void* workspace, size_t ws_bytes, void* stream) {
+  sq_status s = check_mnk(M, N, K);
+  if (s != SQ_OK) return s;
+  if (M == 0) return SQ_OK;
+  if (!q_a || !s_tok || !q_w || !s_ch || !y_bf16) return SQ_ERR_NULL;
+  if (!aligned16(q_a) || !aligned16(s_tok) || !aligned16(q_w) || !aligned16(s_ch) ||
+      !aligned16(y_bf16))
+    return SQ_ERR_ALIGN;
+  return run_gemm(GK_I8_SCALE, q_a, q_w, s_tok, s_ch, nullptr, y_bf16, M, N, K, workspace,
+                  ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+sq_status w8a8_mm_i32(const int8_t* q_a, const int8_t* q_w, int32_t* acc, int64_t M, int64_t N,
+                      int64_t K, void* workspace, size_t ws_bytes, void* stream) {
+  sq_status s = check_mnk(M, N, K);
+  if (s != SQ_OK) return s;
+  if (M == 0) return SQ_OK;
+  if (!q_a || !q_w || !acc) return SQ_ERR_NULL;
+  if (!aligned16(q_a) || !aligned16(q_w) || !aligned16(acc)) return SQ_ERR_ALIGN;
+  return run_gemm(GK_I8_I32, q_a, q_w, nullptr, nullptr, nullptr, acc, M, N, K, workspace,
+                  ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+sq_status w8a8_gs128_mm(const int8_t* q_a, const float* s_tok, const int8_t* q_w,
+                        const float* s_blk, void* y_bf16, int64_t M, int64_t N, int64_t K,
+                        void* workspace, size_t ws_bytes, void* stream) {
+  sq_status s = check_mnk(M, N, K);
+  if (s != SQ_OK) return s;
+  if (M == 0) return SQ_OK;
+  if (!q_a || !s_tok || !q_w || !s_blk || !y_bf16) return SQ_ERR_NULL;
+  if (!aligned16(q_a) || !aligned16(s_tok) || !aligned16(q_w) || !aligned16(s_blk) ||
+      !aligned16(y_bf16))
+    return SQ_ERR_ALIGN;
+  return run_gemm(GK_GS128, q_a, q_w, s_tok, nullptr, s_blk, y_bf16, M, N, K, workspace,
+                  ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+sq_status w8a16_mm(const void* x_bf16, const int8_t* q_w, const float* s_ch, void* y_bf16,
+                   int64_t M, int64_t N, int64_t K, void* workspace, size_t ws_bytes,
+                   void* stream) {
+  sq_status s = check_mnk(M, N, K);
+  if (s != SQ_OK) return s;
+  if (M == 0) return SQ_OK;
+  if (!x_bf16 || !q_w || !s_ch || !y_bf16) return SQ_ERR_NULL;
+  if (!aligned16(x_bf16) || !aligned16(q_w) || !aligned16(s_ch) || !aligned16(y_bf16))
+    return SQ_ERR_ALIGN;
+  const int sms = num_sms();
+  if (sms <= 0) return SQ_ERR_CUDA;
+  size_t w_off = 0;
+  const size_t need = w8a16_ws_bytes(M, N, K, sms, &w_off);
+  if (!workspace || ws_bytes < need) return SQ_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return SQ_ERR_ALIGN;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  __nv_bfloat16* wb = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(workspace) + w_off);
+  const int64_t n16 = N * K / 16;
+  const int64_t blocks = (n16 + 255) / 256 < 4 * sms ? (n16 + 255) / 256 : 4 * sms;
+  i8_to_bf16_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(q_w, wb, n16);
+  if (launch_status() != SQ_OK) return SQ_ERR_CUDA;
+  return run_gemm(GK_BF16, x_bf16, wb, nullptr, s_ch, nullptr, y_bf16, M, N, K, workspace,
+                  w_off, st);
+}
+
+sq_status sq_check_device_error(int reset) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return SQ_ERR_CUDA;
+  unsigned int w = 0;
+  if (cudaMemcpyFromSymbol(&w, g_error_word, sizeof(w)) != cudaSuccess) return SQ_ERR_CUDA;
+  if (reset && w) {
+    const unsigned int z = 0;
+    if (cudaMemcpyToSymbol(g_error_word, &z, sizeof(z)) != cudaSuccess) return SQ_ERR_CUDA;
+  }
+  return (w & kErrTimeout) ? SQ_ERR_TIMEOUT : SQ_OK;
+}
+
+}  // extern "C"
