@@ -98,6 +98,24 @@ sq_status w8a16_mm(const void* x_bf16, const int8_t* q_w, const float* s_ch, voi
                    int64_t M, int64_t N, int64_t K, void* workspace, size_t ws_bytes,
                    void* stream);
 
+/* W8A8 GEMM that allocates nothing and takes no workspace.  The quantisation
+ * pages have no counterpart: this exists for callers that cannot call
+ * cudaMalloc, such as a plugin whose host framework owns all device memory and
+ * passes only inputs and outputs, or a latency-critical thread on which
+ * cudaMalloc would synchronise the device.  Same arguments, arithmetic and
+ * results as w8a8_scaled_mm without the workspace.  For M <= 32 the split-K
+ * partial sums live in a 5 MiB array in the library's static device memory
+ * (held on every GPU that loads the library until the process exits); the
+ * call returns SQ_ERR_WORKSPACE if these sizes would need more than that (not
+ * the case on a 148-SM B200) and SQ_ERR_SHAPE if N > 2,097,152.  The first
+ * call on a device looks up the array's device address (a synchronous runtime
+ * call), so make it before any stream capture.  Every call shares the one
+ * array and clears its counters first: calls that may overlap on the GPU (other
+ * streams, other threads) race and must not be issued. */
+sq_status w8a8_scaled_mm_noalloc(const int8_t* q_a, const float* s_tok, const int8_t* q_w,
+                                 const float* s_ch, void* y_bf16, int64_t M, int64_t N,
+                                 int64_t K, void* stream);
+
 /* Bytes of workspace an operation needs for these sizes (0 = none). */
 size_t sq_workspace_bytes(int op, int64_t M, int64_t N, int64_t K);
 

@@ -60,6 +60,7 @@ def lib() -> ctypes.CDLL:
                 "w8a8_gs128_mm": [vp, vp, vp, vp, vp, i64, i64, i64, vp, sz, vp],
                 "w8a16_mm": [vp, vp, vp, vp, i64, i64, i64, vp, sz, vp],
                 "w8a8_mm_i32": [vp, vp, vp, i64, i64, i64, vp, sz, vp],
+                "w8a8_scaled_mm_noalloc": [vp, vp, vp, vp, vp, i64, i64, i64, vp],
                 "sq_smooth_factors": [vp, i64, vp, i64, i64, dbl, dbl, vp, vp, vp],
                 "sq_quant_weight": [vp, vp, vp, vp, i64, i64, i64, vp],
                 "sq_check_device_error": [ctypes.c_int],
@@ -78,7 +79,7 @@ def lib() -> ctypes.CDLL:
 
 EXPORTS = ("sq_quant_per_token", "w8a8_scaled_mm", "w8a8_gs128_mm", "w8a16_mm",
            "sq_workspace_bytes", "w8a8_mm_i32", "sq_smooth_factors", "sq_quant_weight",
-           "sq_check_device_error", "sq_status_string")
+           "sq_check_device_error", "sq_status_string", "w8a8_scaled_mm_noalloc")
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -142,6 +143,18 @@ def w8a8_scaled_mm(q_a, s_tok, q_w, s_ch, out: Optional[torch.Tensor] = None):
     _check("w8a8_scaled_mm", lib().w8a8_scaled_mm(
         _ptr(q_a), _ptr(s_tok), _ptr(q_w), _ptr(s_ch), _ptr(y), M, N, K, _ptr(ws), wsb,
         _stream(q_a.device)))
+    return y
+
+
+def w8a8_scaled_mm_noalloc(q_a, s_tok, q_w, s_ch, out: Optional[torch.Tensor] = None):
+    """w8a8_scaled_mm without a workspace, for callers that cannot allocate
+    device memory (the library's static scratch holds the split-K partials).
+    Calls must not overlap on the GPU."""
+    M, K = q_a.shape
+    N = q_w.shape[0]
+    y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=q_a.device)
+    _check("w8a8_scaled_mm_noalloc", lib().w8a8_scaled_mm_noalloc(
+        _ptr(q_a), _ptr(s_tok), _ptr(q_w), _ptr(s_ch), _ptr(y), M, N, K, _stream(q_a.device)))
     return y
 
 

@@ -392,3 +392,72 @@ sq_status sq_check_device_error(int reset) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// W8A8 GEMM for callers that cannot allocate device memory.
+//
+// Some callers of this library cannot call cudaMalloc: a plugin whose host
+// framework owns every byte of device memory and hands it only the layer's
+// inputs and outputs, or a latency-critical serving thread where cudaMalloc
+// would synchronise the device and stall other streams.  For the small-token
+// (M <= 32) split-K schedule, the only operation here that needs scratch, this
+// entry point uses a fixed array in the library's own device memory instead
+// of a caller-provided workspace.  The array is a file-scope static, so every
+// GPU that loads the library holds it until the process exits.
+
+namespace {
+// Counter region (64 KiB) + stream-K partial slots for up to 148 CTAs at the
+// widest small-M tile (2 slots x 128 rows x 32 columns x 4 bytes per CTA).
+constexpr size_t kNoAllocScratchBytes = 5u << 20;  // 5 MiB
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+// Device address of g_noalloc_scratch for the current device, looked up once
+// per device (with that device current) and cached.  In host code the
+// symbol's name is only a host-side stand-in, never a device address.
+void* noalloc_scratch_address() {
+  static std::mutex mu;
+  static void* addr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    addr[dev] = p;
+  }
+  return addr[dev];
+}
+}  // namespace
+
+extern "C" sq_status w8a8_scaled_mm_noalloc(const int8_t* q_a, const float* s_tok,
+                                            const int8_t* q_w, const float* s_ch, void* y_bf16,
+                                            int64_t M, int64_t N, int64_t K, void* stream) {
+  sq_status s = check_mnk(M, N, K);
+  if (s != SQ_OK) return s;
+  if (M == 0) return SQ_OK;
+  if (!q_a || !s_tok || !q_w || !s_ch || !y_bf16) return SQ_ERR_NULL;
+  if (!aligned16(q_a) || !aligned16(s_tok) || !aligned16(q_w) || !aligned16(s_ch) ||
+      !aligned16(y_bf16))
+    return SQ_ERR_ALIGN;
+  const int sms = num_sms();
+  if (sms <= 0) return SQ_ERR_CUDA;
+  const GemmPlan p = plan_gemm(GK_I8_SCALE, M, N, K, sms);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (p.ws_bytes == 0)  // large M: this schedule needs no scratch at all
+    return run_gemm(GK_I8_SCALE, q_a, q_w, s_tok, s_ch, nullptr, y_bf16, M, N, K, nullptr, 0,
+                    st);
+  if (p.ws_bytes > kNoAllocScratchBytes) return SQ_ERR_WORKSPACE;
+  if (static_cast<int64_t>(p.tiles_r) * p.tiles_c > kMaxCounterTiles) return SQ_ERR_SHAPE;
+  void* scratch = noalloc_scratch_address();
+  if (!scratch) return SQ_ERR_CUDA;
+  // The array keeps whatever the previous call left; the arrival counters
+  // must start at zero, so clear the ones this call uses.
+  if (cudaMemsetAsync(scratch, 0, static_cast<size_t>(p.tiles_r) * p.tiles_c * 4, st) !=
+      cudaSuccess)
+    return SQ_ERR_CUDA;
+  return run_gemm(GK_I8_SCALE, q_a, q_w, s_tok, s_ch, nullptr, y_bf16, M, N, K, scratch,
+                  kNoAllocScratchBytes, st);
+}
