@@ -135,6 +135,32 @@ def time_batches(fn, iters, warmup=3):
     return a.elapsed_time(b) / iters * 1e-3
 
 
+def time_graph(fn, calls, reps=5):
+    """Device time per call of fn, with `calls` calls captured in one CUDA graph
+    (so host launch overhead is not measured) and the graph replayed `reps`
+    times back to back."""
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):           # eager warm-up on the capture stream:
+        for i in range(3):               # creates its workspace, sets attributes
+            fn(i)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for i in range(calls):
+            fn(i)
+    g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        g.replay()
+    b.record()
+    torch.cuda.synchronize()
+    del g
+    return a.elapsed_time(b) / (reps * calls) * 1e-3
+
+
 def dist_info():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -207,11 +233,18 @@ def main():
     ap.add_argument("--no-variants", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--profile", choices=["w8a8", "gs128", "w8a16"], default=None,
+                    help="run one operation at --M/--N/--K for --steps calls (for ncu)")
+    ap.add_argument("--M", type=int, default=4096)
+    ap.add_argument("--N", type=int, default=34816)
+    ap.add_argument("--K", type=int, default=5120)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     peaks = load_peaks()
     if args.impl == "reference":
         return reference_arm(args, peaks)
+    if args.profile:
+        return profile_case(args)
 
     import w8a8_int8_quantized_sq_b200 as sq
     from w8a8_int8_quantized_sq_b200 import inputs
@@ -352,6 +385,38 @@ def main():
     return 0
 
 
+def profile_case(args):
+    """One operation at the given sizes, warm-up then --steps timed calls."""
+    import w8a8_int8_quantized_sq_b200 as sq
+    from w8a8_int8_quantized_sq_b200 import inputs
+    dev = torch.device("cuda", 0)
+    M, N, K = args.M, args.N, args.K
+    x = inputs.gen_x(M, K, inputs.SEED_BASE + 100,
+                     inputs.XRecipe(col_count=max(1, K // 100), col_factor=30.0)).to(dev)
+    w = inputs.gen_w(N, K, inputs.SEED_BASE + 100).to(dev)
+    if args.profile == "w8a8":
+        s, inv = sq.smooth_factors(x, w)
+        q_w, s_ch = sq.quant_weight(w, s)
+        fn = lambda: sq.linear_w8a8(x, inv, q_w, s_ch)  # noqa: E731
+    elif args.profile == "gs128":
+        q_w, s_blk = sq.quant_weight(w, None, group=128)
+        q_a, s_tok = sq.quant_per_token(x, None)
+        fn = lambda: sq.w8a8_gs128_mm(q_a, s_tok, q_w, s_blk)  # noqa: E731
+    else:
+        q_w, s_ch = sq.quant_weight(w, None)
+        fn = lambda: sq.w8a16_mm(x, q_w, s_ch)  # noqa: E731
+    del w
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    t_eager = time_batches(lambda i: fn(), args.steps, warmup=0)
+    t_graph = time_graph(lambda i: fn(), args.steps, reps=3)
+    print(json.dumps({"profile": args.profile, "M": M, "N": N, "K": K, "steps": args.steps,
+                      "ms_per_call": t_graph * 1e3, "ms_per_call_eager": t_eager * 1e3}),
+          flush=True)
+    return 0
+
+
 def variants(sq, inputs, dev, peaks):
     """The other workloads, each timed alone with enough weight copies to exceed L2."""
     out = []
@@ -367,16 +432,19 @@ def variants(sq, inputs, dev, peaks):
     del w
     copies = max(2, -(-3 * l2 // q_w.numel()))
     qws = [q_w.clone() for _ in range(copies)]
-    t = time_batches(lambda i: sq.linear_w8a8(x, inv, qws[i % copies], s_ch), 60)
-    tg = time_batches(lambda i: sq.w8a8_scaled_mm(*sq.quant_per_token(x, inv), qws[i % copies],
-                                                  s_ch), 60)
+    t = time_graph(lambda i: sq.linear_w8a8(x, inv, qws[i % copies], s_ch), 4 * copies)
+    q_a, s_tok = sq.quant_per_token(x, inv)
+    tg = time_graph(lambda i: sq.w8a8_scaled_mm(q_a, s_tok, qws[i % copies], s_ch), 4 * copies)
+    tq = time_graph(lambda i: sq.quant_per_token(x, inv), 4 * copies)
     byt = algo_bytes_quant(wl.M, wl.K) + algo_bytes_w8a8(wl.M, wl.N, wl.K)
     out.append({"workload": wl.name, "metric": "GB/s (quant + GEMM, algorithmic bytes)",
                 "value": byt / t / 1e9, "unit": "GB/s", "us_per_call": t * 1e6,
                 "frac_of_hbm": byt / t / 1e9 / hbm, "tokens_per_s": wl.M / t,
                 "tops": 2.0 * wl.M * wl.N * wl.K / t / 1e12, "weight_copies": copies,
-                "us_per_call_recheck": tg * 1e6})
-    del qws, q_w, x
+                "gemm_us": tg * 1e6, "quant_us": tq * 1e6,
+                "gemm_frac_of_hbm": algo_bytes_w8a8(wl.M, wl.N, wl.K) / tg / 1e9 / hbm,
+                "timing": "CUDA graph of back-to-back calls, rotating weight copies"})
+    del qws, q_w, x, q_a
 
     # gs128 W8A8 (M=2048)
     wl = inputs.workload(3)
@@ -387,9 +455,9 @@ def variants(sq, inputs, dev, peaks):
     q_a, s_tok = sq.quant_per_token(x, None)
     copies = max(2, -(-3 * l2 // (q_w.numel() + q_a.numel())))
     sets = [(q_a.clone(), q_w.clone()) for _ in range(copies)]
-    t = time_batches(lambda i: sq.w8a8_gs128_mm(sets[i % copies][0], s_tok, sets[i % copies][1],
-                                                s_blk), 30)
-    tq = time_batches(lambda i: sq.quant_per_token(x, None), 30)
+    t = time_graph(lambda i: sq.w8a8_gs128_mm(sets[i % copies][0], s_tok, sets[i % copies][1],
+                                              s_blk), 2 * copies)
+    tq = time_graph(lambda i: sq.quant_per_token(x, None), 2 * copies)
     ops = 2.0 * wl.M * wl.N * wl.K
     int8_peak = peaks["bf16_tflops"] * INT8_PER_BF16
     out.append({"workload": wl.name, "metric": "TOPS (gs128 GEMM)", "value": ops / t / 1e12,
@@ -408,7 +476,7 @@ def variants(sq, inputs, dev, peaks):
     for M in inputs.W8A16_M_VALUES:
         x = wl.make_x(M).to(dev)
         if M <= 16:
-            t = time_batches(lambda i: sq.w8a16_mm(x, qws[i % copies], s_ch), 60)
+            t = time_graph(lambda i: sq.w8a16_mm(x, qws[i % copies], s_ch), 4 * copies)
             byt = algo_bytes_w8a16(M, wl.N, wl.K)
             out.append({"workload": f"{wl.name}_M{M}", "metric": "GB/s (algorithmic bytes)",
                         "value": byt / t / 1e9, "unit": "GB/s", "us_per_call": t * 1e6,

@@ -78,6 +78,18 @@ sq_status w8a8_scaled_mm(const int8_t* q_a, const float* s_tok, const int8_t* q_
                          const float* s_ch, void* y_bf16, int64_t M, int64_t N, int64_t K,
                          void* workspace, size_t ws_bytes, void* stream);
 
+/* The whole W8A8 linear layer in one call [P1, P4]: sq_quant_per_token of x
+ * into the caller's q_a (int8 [M,K]) and s_tok (fp32 [M]), then
+ * w8a8_scaled_mm into y.  The GEMM is launched as a programmatic dependent of
+ * the quantisation kernel: it may start, allocate tensor memory and begin
+ * streaming q_w while the quantisation still runs, and reads q_a, s_tok only
+ * after that kernel has completed.  q_w and s_ch must therefore not be written
+ * by that quantisation (they are inputs of this call; nothing else runs in
+ * between).  Workspace as for w8a8_scaled_mm (SQ_OP_W8A8). */
+sq_status sq_w8a8_linear(const void* x_bf16, const float* inv_smooth, const int8_t* q_w,
+                         const float* s_ch, void* y_bf16, int8_t* q_a, float* s_tok, int64_t M,
+                         int64_t N, int64_t K, void* workspace, size_t ws_bytes, void* stream);
+
 /* W8A8 with group-size-128 weight scales [P5]: s_blk fp32 [N, K/128], one
  * scale per (output row, 128-wide K block).  With P_kb[m,n] the exact int32
  * partial over block kb:  acc = 0; for kb ascending:

@@ -208,7 +208,8 @@ def test_w8a16_prefill_sampled_rows():
     _check_w8a16(d["x"], d["q_w"], d["s_ch"], rows=rows)
 
 
-@pytest.mark.parametrize("M,N,K", [(3, 144, 256), (33, 256, 640)])
+@pytest.mark.parametrize("M,N,K", [(3, 144, 256), (17, 144, 384), (32, 256, 1280),
+                                   (8, 5120, 5120), (33, 256, 640)])
 def test_w8a16_shapes(M, N, K):
     x = inputs.gen_x(M, K, 5)
     q_w = torch.randint(-127, 128, (N, K), dtype=torch.int8)
@@ -249,3 +250,18 @@ def test_error_codes():
     # M = 0 is a no-op
     assert L.w8a8_scaled_mm(None, None, None, None, None, 0, 32, 256, None, 0, None) == 0
     sq.check_device_error()
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 128, 256), (8, 5120, 5120), (33, 256, 640), (300, 512, 1024)])
+def test_fused_linear_pdl(M, N, K):
+    """sq_w8a8_linear (quant, then the GEMM as a programmatic dependent)."""
+    x = inputs.gen_x(M, K, 17, inputs.XRecipe(col_count=2, col_factor=30.0))
+    w = inputs.gen_w(N, K, 17)
+    s, inv = oracle.smooth_factors(x, w)
+    q_w, s_ch = oracle.quant_weight(w, s)
+    q_a, s_tok = oracle.quant_per_token(x, inv)
+    ref = oracle.w8a8_scaled_mm(q_a, s_tok, q_w, s_ch)
+    xd, invd, qwd, schd = x.cuda(), inv.cuda(), q_w.cuda(), s_ch.cuda()
+    for _ in range(3):  # back-to-back calls overlap one call's GEMM with the next quant
+        y = sq.linear_w8a8(xd, invd, qwd, schd)
+    assert_same(y, ref, "fused linear")

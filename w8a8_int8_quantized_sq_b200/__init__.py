@@ -61,6 +61,7 @@ def lib() -> ctypes.CDLL:
                 "w8a16_mm": [vp, vp, vp, vp, i64, i64, i64, vp, sz, vp],
                 "w8a8_mm_i32": [vp, vp, vp, i64, i64, i64, vp, sz, vp],
                 "w8a8_scaled_mm_noalloc": [vp, vp, vp, vp, vp, i64, i64, i64, vp],
+                "sq_w8a8_linear": [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, vp, sz, vp],
                 "sq_smooth_factors": [vp, i64, vp, i64, i64, dbl, dbl, vp, vp, vp],
                 "sq_quant_weight": [vp, vp, vp, vp, i64, i64, i64, vp],
                 "sq_check_device_error": [ctypes.c_int],
@@ -79,7 +80,8 @@ def lib() -> ctypes.CDLL:
 
 EXPORTS = ("sq_quant_per_token", "w8a8_scaled_mm", "w8a8_gs128_mm", "w8a16_mm",
            "sq_workspace_bytes", "w8a8_mm_i32", "sq_smooth_factors", "sq_quant_weight",
-           "sq_check_device_error", "sq_status_string", "w8a8_scaled_mm_noalloc")
+           "sq_check_device_error", "sq_status_string", "w8a8_scaled_mm_noalloc",
+           "sq_w8a8_linear")
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -189,10 +191,19 @@ def w8a16_mm(x, q_w, s_ch):
     return y
 
 
-def linear_w8a8(x, inv_s, q_w, s_ch):
-    """y = W8A8 linear layer: per-token quant with the 1/s fold, then the GEMM."""
-    q_a, s_tok = quant_per_token(x, inv_s)
-    return w8a8_scaled_mm(q_a, s_tok, q_w, s_ch)
+def linear_w8a8(x, inv_s, q_w, s_ch, out: Optional[torch.Tensor] = None):
+    """y = W8A8 linear layer in one call (sq_w8a8_linear): per-token quant with
+    the 1/s fold, then the GEMM launched as a programmatic dependent."""
+    M, K = x.shape
+    N = q_w.shape[0]
+    q_a = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    s_tok = torch.empty((M,), dtype=torch.float32, device=x.device)
+    y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    ws, wsb = workspace(OP_W8A8, M, N, K, x.device)
+    _check("sq_w8a8_linear", lib().sq_w8a8_linear(
+        _ptr(x), _ptr(inv_s), _ptr(q_w), _ptr(s_ch), _ptr(y), _ptr(q_a), _ptr(s_tok), M, N, K,
+        _ptr(ws), wsb, _stream(x.device)))
+    return y
 
 
 def smooth_factors(x, w, cap: float = 16.0, floor: float = 1e-5):

@@ -30,6 +30,7 @@
 // the buffer's starting pattern for its next use.
 #pragma once
 #include "ptx.cuh"
+#include "quant.cuh"  // exact int8 -> bf16 conversion
 
 namespace sq {
 
@@ -56,30 +57,58 @@ __host__ __device__ constexpr int pow2_at_least(int v) {
   return p;
 }
 
-template <bool I8_, int BN_, int STAGES_, bool SWAP_, int EPI_>
+// CONV_ = true (the W8A16 dequant-on-load path): operand A arrives as int8
+// weight rows, RK K blocks per raw shared-memory stage (TMA, 128-byte
+// swizzle).  Eight converter warps expand a whole raw stage exactly to bf16
+// and write it straight into a ring of STAGES A tiles in tensor memory
+// (tcgen05.st; 32 columns of two bf16 per 128-lane row), then wait for their
+// stores once and release the raw stage; the MMA reads A from tensor memory.
+// A second producer thread loads each K block's B tile directly into a
+// shared-memory ring that shadows the A ring, so the raw ring can be deeper
+// than the A ring: the raw loads stay in flight while a stage is converted.  Keeping A out of shared
+// memory leaves 2 bytes of shared-memory traffic per weight byte instead of 6.
+template <bool I8_, int BN_, int STAGES_, bool SWAP_, int EPI_, bool CONV_ = false,
+          int RSTAGES_ = 0>
 struct GemmCfg {
   static constexpr bool I8 = I8_;
   static constexpr int BN = BN_;
   static constexpr int STAGES = STAGES_;
   static constexpr bool SWAP = SWAP_;
   static constexpr int EPI = EPI_;
+  static constexpr bool CONV = CONV_;
+  static constexpr int RSTAGES = CONV_ ? RSTAGES_ : 0;
   static constexpr int BM = 128;
   static constexpr int KB_BYTES = 128;
   static constexpr int KB_ELEMS = I8 ? 128 : 64;
   static constexpr int A_BYTES = BM * KB_BYTES;
   static constexpr int B_BYTES = BN * KB_BYTES;
+  // raw stage: RK K blocks of int8 weight rows, as RK/2 boxes of 128 rows x
+  // 128 bytes (two K blocks per row, 128-byte swizzle), then the RK B tiles
+  static constexpr int RK = 4;
+  static constexpr int RAW_BOX_BYTES = BM * 128;
+  static constexpr int RAW_A_BYTES = (RK / 2) * RAW_BOX_BYTES;
+  static constexpr int RAW_BYTES = RAW_A_BYTES;
   static constexpr int NE = (EPI == EPI_GS128) ? 8 : 4;  // epilogue warps
-  static constexpr int THREADS = 64 + NE * 32;
+  static constexpr int NCV = CONV ? 8 : 0;               // converter warps (2 per row)
+  static constexpr int THREADS = 64 + NE * 32 + NCV * 32;
   static constexpr int NACC = (EPI == EPI_GS128) ? 4 : 2;
-  static constexpr int TMEM_COLS = pow2_at_least(NACC * BN);
+  // Narrow (swapped, small-token) tiles rotate the K blocks over NSUB
+  // independent accumulators, so consecutive tiny MMAs do not wait on each
+  // other's result; the epilogue adds them in a fixed order.
+  static constexpr int NSUB = (SWAP && EPI != EPI_GS128) ? 4 : 1;
+  static constexpr int ACC_COLS = NACC * NSUB * BN;
+  static constexpr int A_TMEM_COLS = 32;  // one 128 x 64 bf16 A tile in tensor memory
+  static constexpr int TMEM_COLS = CONV ? 512 : pow2_at_least(ACC_COLS);
   static constexpr int CW = BN < 32 ? BN : 32;  // columns per tcgen05.ld
   static constexpr int CPT = BN / (NE / 4);     // columns owned by one epilogue thread
   static constexpr int SBLK_STRIDE = BN + 4;    // floats per K block in the staged s_blk
   // shared memory carve-up (offsets from a 1024-byte aligned base)
-  static constexpr int OFF_A = 0;
-  static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
+  static constexpr int A_SMEM_BYTES = CONV ? 0 : A_BYTES;  // CONV: A lives in TMEM
+  static constexpr int OFF_RAW = 0;
+  static constexpr int OFF_A = OFF_RAW + RSTAGES * RAW_BYTES;
+  static constexpr int OFF_B = OFF_A + STAGES * A_SMEM_BYTES;
   static constexpr int OFF_BAR = OFF_B + STAGES * B_BYTES;
-  static constexpr int NUM_BARS = 2 * STAGES + 2 * NACC + 1;
+  static constexpr int NUM_BARS = 2 * STAGES + 2 * NACC + 1 + 2 * RSTAGES;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int OFF_SBLK = (OFF_MISC + 16 + 15) / 16 * 16;
   static constexpr int smem_bytes(int kb_total) {
@@ -87,6 +116,10 @@ struct GemmCfg {
   }
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N for M = 128");
   static_assert(EPI != EPI_GS128 || (I8 && !SWAP && BN % 64 == 0), "gs128 layout");
+  static_assert(!CONV || (!I8 && SWAP && EPI == EPI_SCALE), "dequant-on-load is W8A16, swapped");
+  static_assert(!CONV || (RAW_BYTES % 1024 == 0 && B_BYTES % 16 == 0), "raw stage alignment");
+  static_assert(!CONV || ACC_COLS + STAGES * A_TMEM_COLS <= 512, "tensor memory A ring");
+
   static_assert(TMEM_COLS <= 512, "tensor memory");
 };
 
@@ -212,6 +245,25 @@ __device__ __forceinline__ void tmem_ld_chunk(uint32_t taddr, uint32_t (&v)[Cfg:
   else tmem_ld16(taddr, v);
 }
 
+// Columns [c, c + CW) of an accumulator made of `nsub` sub-accumulators
+// (BN columns apart), summed in sub-accumulator order.
+template <class Cfg>
+__device__ __forceinline__ void tmem_ld_acc(uint32_t tb, int c, int nsub,
+                                            uint32_t (&v)[Cfg::CW]) {
+  tmem_ld_chunk<Cfg>(tb + c, v);
+  for (int sub = 1; sub < nsub; ++sub) {
+    uint32_t t[Cfg::CW];
+    tmem_ld_chunk<Cfg>(tb + sub * Cfg::BN + c, t);
+#pragma unroll
+    for (int j = 0; j < Cfg::CW; ++j) {
+      if constexpr (Cfg::I8)
+        v[j] = static_cast<uint32_t>(static_cast<int32_t>(v[j]) + static_cast<int32_t>(t[j]));
+      else
+        v[j] = __float_as_uint(__fadd_rn(__uint_as_float(v[j]), __uint_as_float(t[j])));
+    }
+  }
+}
+
 // ------------------------------------------------------------------ kernel
 template <class Cfg>
 __global__ void __launch_bounds__(Cfg::THREADS, 1)
@@ -230,6 +282,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   uint64_t* tfull = bars + 2 * STAGES;
   uint64_t* tempty = tfull + NACC;
   uint64_t* drain = tempty + NACC;
+  uint64_t* raw_full = drain + 1;             // CONV: producer -> converters
+  uint64_t* raw_empty = raw_full + Cfg::RSTAGES;  // CONV: converters -> producer
+  uint8_t* smRaw = smem + Cfg::OFF_RAW;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::OFF_MISC + 4);
   volatile int* sk_flag = reinterpret_cast<volatile int*>(smem + Cfg::OFF_MISC + 8);
@@ -248,6 +303,16 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       mbar_init(tempty + a, NE);
     }
     mbar_init(drain, 1);
+    if constexpr (Cfg::CONV) {
+      // the converted stage completes on the converter warps' arrivals plus
+      // the B tile's transaction bytes
+      // converted stage: converter warps' arrivals + the producer's B tile
+      for (int s = 0; s < STAGES; ++s) mbar_init(full + s, Cfg::NCV + 1);
+      for (int s = 0; s < Cfg::RSTAGES; ++s) {
+        mbar_init(raw_full + s, 1);
+        mbar_init(raw_empty + s, Cfg::NCV);
+      }
+    }
     *abort_flag = 0;
     *sk_flag = 0;
     fence_mbar_init();
@@ -261,7 +326,145 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
-  if (warp == 0) {
+  if (warp == 0 && Cfg::CONV) {
+    // ------------------------------- TMA producers: raw int8 weights (lane 0)
+    //                                   and the K blocks' B tiles (lane 1)
+    if (lane == 0) {
+      tma_prefetch_desc(&tmA);
+      uint32_t rs = 0, rph = 0;
+      long long fills = 0;
+      SegIter it;
+      it.init(g);
+      Seg s;
+      bool ok = true;
+      while (ok && it.next(g, s)) {
+        const int rt = s.tile % g.tiles_r;
+        for (int kb = s.kb0; kb < s.kb1; kb += Cfg::RK) {
+          const int n = s.kb1 - kb < Cfg::RK ? s.kb1 - kb : Cfg::RK;  // K blocks used
+          if (!wait_bounded(raw_empty + rs, rph ^ 1u, abort_flag)) { ok = false; break; }
+          uint8_t* st = smRaw + rs * Cfg::RAW_BYTES;
+          const int boxes = (n + 1) / 2;
+          mbar_arrive_expect_tx(raw_full + rs, boxes * Cfg::RAW_BOX_BYTES);
+          // 128 contiguous weight bytes per row per box, both boxes back to back
+          for (int b2 = 0; b2 < boxes; ++b2)
+            tma_load_2d(st + b2 * Cfg::RAW_BOX_BYTES, &tmA, (kb + 2 * b2) * Cfg::KB_ELEMS,
+                        rt * Cfg::BM, raw_full + rs);
+          ++fills;
+          if (++rs == Cfg::RSTAGES) { rs = 0; rph ^= 1u; }
+        }
+      }
+      for (int st = 0; st < Cfg::RSTAGES; ++st) {
+        const long long n = fills / Cfg::RSTAGES + (st < fills % Cfg::RSTAGES ? 1 : 0);
+        if (n > 0) wait_drain(raw_full + st, static_cast<uint32_t>((n - 1) & 1));
+      }
+    } else if (lane == 1) {
+      tma_prefetch_desc(&tmB);
+      griddep_wait();  // the activations may come from the preceding kernel
+      uint32_t cs = 0, cph = 0;
+      long long bfills = 0;
+      SegIter it;
+      it.init(g);
+      Seg s;
+      bool ok = true;
+      while (ok && it.next(g, s)) {
+        const int ct = s.tile / g.tiles_r;
+        for (int kb = s.kb0; kb < s.kb1; ++kb) {
+          if (!wait_bounded(empty + cs, cph ^ 1u, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(full + cs, Cfg::B_BYTES);
+          tma_load_2d(smB + cs * Cfg::B_BYTES, &tmB, kb * Cfg::KB_ELEMS, ct * BN, full + cs);
+          ++bfills;
+          if (++cs == STAGES) { cs = 0; cph ^= 1u; }
+        }
+      }
+      for (int st = 0; st < STAGES; ++st) {
+        const long long n = bfills / STAGES + (st < bfills % STAGES ? 1 : 0);
+        if (n > 0) wait_drain(full + st, static_cast<uint32_t>((n - 1) & 1));
+      }
+    }
+  } else if (warp >= 2 + NE) {
+    // ------------------------------------------- converter warps (CONV only)
+    if constexpr (Cfg::CONV) {
+      const int q = warp & 3;                  // TMEM lane quadrant of this warp
+      const int row = q * 32 + lane;           // weight row of the K block (= TMEM lane)
+      const int half = (warp - (2 + NE)) >> 2; // which 32 of its 64 codes
+      const uint32_t a_lane = tmem + (static_cast<uint32_t>(q * 32) << 16) + Cfg::ACC_COLS;
+      uint32_t rs = 0, rph = 0, cs = 0, cph = 0;
+      SegIter it;
+      it.init(g);
+      Seg s;
+      bool ok = true;
+      while (ok && it.next(g, s)) {
+        for (int kb = s.kb0; kb < s.kb1 && ok; kb += Cfg::RK) {
+          const int n = s.kb1 - kb < Cfg::RK ? s.kb1 - kb : Cfg::RK;
+          if (!wait_bounded(raw_full + rs, rph, abort_flag)) { ok = false; break; }
+          // the A slots of these K blocks are free once the MMAs that read them are done
+          {
+            uint32_t c2 = cs, p2 = cph;
+            for (int c = 0; c < n && ok; ++c) {
+              if (!wait_bounded(empty + c2, p2 ^ 1u, abort_flag)) ok = false;
+              if (++c2 == STAGES) { c2 = 0; p2 ^= 1u; }
+            }
+            if (!ok) break;
+          }
+          tc_fence_after();
+          const uint8_t* raw = smRaw + rs * Cfg::RAW_BYTES;
+          // raw row (128-byte swizzle): K block c is chunks 4(c&1)..4(c&1)+3 of
+          // its box row, 16-byte chunk j at position j ^ (row & 7).  This
+          // thread converts chunks 2*half, 2*half+1 (32 codes -> 32 bf16, two
+          // per column, lower K in the low half) into TMEM columns 16*half ..
+          // 16*half+15 of the K block's A slot.
+          auto chunk = [&](int c, int jj) {
+            return *reinterpret_cast<const uint4*>(
+                raw + (c >> 1) * Cfg::RAW_BOX_BYTES + row * 128 +
+                (((4 * (c & 1) + 2 * half + jj) ^ (row & 7)) << 4));
+          };
+          auto convert = [&](const uint4 w0, const uint4 w1, uint32_t slot) {
+            uint32_t o[16];
+            i8x4_to_bf16x4(w0.x, o[0], o[1]);
+            i8x4_to_bf16x4(w0.y, o[2], o[3]);
+            i8x4_to_bf16x4(w0.z, o[4], o[5]);
+            i8x4_to_bf16x4(w0.w, o[6], o[7]);
+            i8x4_to_bf16x4(w1.x, o[8], o[9]);
+            i8x4_to_bf16x4(w1.y, o[10], o[11]);
+            i8x4_to_bf16x4(w1.z, o[12], o[13]);
+            i8x4_to_bf16x4(w1.w, o[14], o[15]);
+            tmem_st16(a_lane + slot * Cfg::A_TMEM_COLS + half * 16, o);
+          };
+          if (n == Cfg::RK) {
+            uint4 w[Cfg::RK][2];
+#pragma unroll
+            for (int c = 0; c < Cfg::RK; ++c) {  // all loads first
+              w[c][0] = chunk(c, 0);
+              w[c][1] = chunk(c, 1);
+            }
+#pragma unroll
+            for (int c = 0; c < Cfg::RK; ++c)
+              convert(w[c][0], w[c][1], cs + c >= STAGES ? cs + c - STAGES : cs + c);
+          } else {
+            uint32_t c2 = cs;
+            for (int c = 0; c < n; ++c) {
+              convert(chunk(c, 0), chunk(c, 1), c2);
+              if (++c2 == STAGES) c2 = 0;
+            }
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(raw_empty + rs);
+            for (int c = 0; c < n; ++c) {
+              mbar_arrive(full + cs);
+              if (++cs == STAGES) { cs = 0; cph ^= 1u; }
+            }
+          } else {
+            for (int c = 0; c < n; ++c)
+              if (++cs == STAGES) { cs = 0; cph ^= 1u; }
+          }
+          if (++rs == Cfg::RSTAGES) { rs = 0; rph ^= 1u; }
+        }
+      }
+    }
+  } else if (warp == 0) {
     // ------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&tmA);
@@ -272,17 +475,46 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       it.init(g);
       Seg s;
       bool ok = true;
+      // The weight operand (A when SWAP, else B) of the first STAGES fills is
+      // requested before griddep_wait, so that under a programmatic launch the
+      // weight stream starts while the preceding kernel still produces the
+      // activations; their activation tiles follow right after the wait.
+      bool waited = false;
+      int pend_kb[STAGES], pend_row[STAGES];
+      auto act_load = [&](int st, int kb, int row) {
+        if constexpr (Cfg::SWAP)
+          tma_load_2d(smB + st * Cfg::B_BYTES, &tmB, kb * Cfg::KB_ELEMS, row, full + st);
+        else
+          tma_load_2d(smA + st * Cfg::A_BYTES, &tmA, kb * Cfg::KB_ELEMS, row, full + st);
+      };
+      auto release_pending = [&]() {
+        griddep_wait();
+        const int n = fills < STAGES ? static_cast<int>(fills) : STAGES;
+        for (int i = 0; i < n; ++i) act_load(i, pend_kb[i], pend_row[i]);
+        waited = true;
+      };
       while (ok && it.next(g, s)) {
         const int rt = s.tile % g.tiles_r, ct = s.tile / g.tiles_r;
         for (int kb = s.kb0; kb < s.kb1; ++kb) {
+          if (!waited && fills == STAGES) release_pending();
           if (!wait_bounded(empty + stage, phase ^ 1u, abort_flag)) {
             ok = false;
             break;
           }
           mbar_arrive_expect_tx(full + stage, Cfg::A_BYTES + Cfg::B_BYTES);
-          tma_load_2d(smA + stage * Cfg::A_BYTES, &tmA, kb * Cfg::KB_ELEMS, rt * Cfg::BM,
-                      full + stage);
-          tma_load_2d(smB + stage * Cfg::B_BYTES, &tmB, kb * Cfg::KB_ELEMS, ct * BN, full + stage);
+          const int act_row = Cfg::SWAP ? ct * BN : rt * Cfg::BM;
+          if constexpr (Cfg::SWAP)
+            tma_load_2d(smA + stage * Cfg::A_BYTES, &tmA, kb * Cfg::KB_ELEMS, rt * Cfg::BM,
+                        full + stage);
+          else
+            tma_load_2d(smB + stage * Cfg::B_BYTES, &tmB, kb * Cfg::KB_ELEMS, ct * BN,
+                        full + stage);
+          if (waited) {
+            act_load(stage, kb, act_row);
+          } else {
+            pend_kb[fills] = kb;
+            pend_row[fills] = act_row;
+          }
           ++fills;
           if (++stage == STAGES) {
             stage = 0;
@@ -290,6 +522,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           }
         }
       }
+      if (!waited) release_pending();
       // no copy may still be writing shared memory when the CTA exits
       for (int st = 0; st < STAGES; ++st) {
         const long long n = fills / STAGES + (st < fills % STAGES ? 1 : 0);
@@ -328,16 +561,20 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           const uint32_t a = local % NACC, u = local / NACC;
           if (!wait_bounded(tempty + a, (u & 1u) ^ 1u, abort_flag)) break;
           tc_fence_after();
-          const uint32_t d = tmem + a * BN;
           for (int kb = s.kb0; kb < s.kb1; ++kb) {
             if (!wait_bounded(full + stage, phase, abort_flag)) { ok = false; break; }
             tc_fence_after();
             const uint32_t sa = smem_u32(smA + stage * Cfg::A_BYTES);
             const uint32_t sb = smem_u32(smB + stage * Cfg::B_BYTES);
+            const int i = kb - s.kb0;
+            const uint32_t d = tmem + (a * Cfg::NSUB + i % Cfg::NSUB) * BN;
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-              const uint32_t accum = (kb > s.kb0 || k > 0) ? 1u : 0u;
-              if constexpr (Cfg::I8)
+              const uint32_t accum = (i >= Cfg::NSUB || k > 0) ? 1u : 0u;
+              if constexpr (Cfg::CONV)
+                mma_bf16_tmem_a(d, tmem + Cfg::ACC_COLS + stage * Cfg::A_TMEM_COLS + k * 8,
+                                smem_desc_sw128(sb + k * 32), idesc, accum);
+              else if constexpr (Cfg::I8)
                 mma_i8(d, smem_desc_sw128(sa + k * 32), smem_desc_sw128(sb + k * 32), idesc, accum);
               else
                 mma_bf16(d, smem_desc_sw128(sa + k * 32), smem_desc_sw128(sb + k * 32), idesc,
@@ -358,6 +595,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
+    griddep_wait();  // the scales may come from the preceding kernel
     const int ew = warp - 2;
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
     const int rr = q * 32 + lane;
@@ -447,12 +685,13 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         if (named_bar_or(1, nthr, !w_ok)) break;
         tc_fence_after();
         const int rt = s.tile % g.tiles_r, ct = s.tile / g.tiles_r;
-        const uint32_t tb = lane_base + a * BN;
+        const uint32_t tb = lane_base + a * Cfg::NSUB * BN;
+        const int nsub = s.kb1 - s.kb0 < Cfg::NSUB ? s.kb1 - s.kb0 : Cfg::NSUB;
         if (s.kb0 == 0 && s.kb1 == g.kb_total) {
 #pragma unroll 1
           for (int c = 0; c < BN; c += CW) {
             uint32_t v[CW];
-            tmem_ld_chunk<Cfg>(tb + c, v);
+            tmem_ld_acc<Cfg>(tb, c, nsub, v);
             store_chunk<Cfg>(g, rt, ct, rr, c, v);
           }
         } else {
@@ -465,7 +704,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
 #pragma unroll 1
           for (int c = 0; c < BN; c += CW) {
             uint32_t v[CW];
-            tmem_ld_chunk<Cfg>(tb + c, v);
+            tmem_ld_acc<Cfg>(tb, c, nsub, v);
 #pragma unroll
             for (int j = 0; j < CW; j += 4)
               *reinterpret_cast<uint4*>(wrow + c + j) = make_uint4(v[j], v[j + 1], v[j + 2], v[j + 3]);
@@ -486,23 +725,40 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
               uint32_t v[CW];
 #pragma unroll
               for (int j = 0; j < CW; ++j) v[j] = 0u;
-              for (long long b = b_lo; b <= b_hi; ++b) {
-                const int sl = sk_start(b, G, T) >= it0 ? 0 : 1;
-                const uint32_t* prow =
-                    g.ws + (static_cast<size_t>(b * 2 + sl) * Cfg::BM + rr) * BN + c;
+              // parts are summed in CTA order; up to NB parts' loads in flight
+              constexpr int NB = CW >= 32 ? 2 : 4;
+              for (long long b0 = b_lo; b0 <= b_hi; b0 += NB) {
+                int4 w[NB][CW / 4];
 #pragma unroll
-                for (int j = 0; j < CW; j += 4) {
-                  const int4 w = ld_cg_v4(prow + j);
-                  const uint32_t wv[4] = {static_cast<uint32_t>(w.x), static_cast<uint32_t>(w.y),
-                                          static_cast<uint32_t>(w.z), static_cast<uint32_t>(w.w)};
+                for (int u = 0; u < NB; ++u) {
+                  const long long b = b0 + u;
+                  if (b <= b_hi) {
+                    const int sl = sk_start(b, G, T) >= it0 ? 0 : 1;
+                    const uint32_t* prow =
+                        g.ws + (static_cast<size_t>(b * 2 + sl) * Cfg::BM + rr) * BN + c;
 #pragma unroll
-                  for (int i = 0; i < 4; ++i) {
-                    if constexpr (Cfg::I8)
-                      v[j + i] = static_cast<uint32_t>(static_cast<int32_t>(v[j + i]) +
-                                                       static_cast<int32_t>(wv[i]));
-                    else
-                      v[j + i] = __float_as_uint(__fadd_rn(__uint_as_float(v[j + i]),
-                                                           __uint_as_float(wv[i])));
+                    for (int j = 0; j < CW / 4; ++j) w[u][j] = ld_cg_v4(prow + 4 * j);
+                  }
+                }
+#pragma unroll
+                for (int u = 0; u < NB; ++u) {
+                  if (b0 + u <= b_hi) {
+#pragma unroll
+                    for (int j = 0; j < CW / 4; ++j) {
+                      const uint32_t wv[4] = {
+                          static_cast<uint32_t>(w[u][j].x), static_cast<uint32_t>(w[u][j].y),
+                          static_cast<uint32_t>(w[u][j].z), static_cast<uint32_t>(w[u][j].w)};
+#pragma unroll
+                      for (int i = 0; i < 4; ++i) {
+                        uint32_t& acc = v[4 * j + i];
+                        if constexpr (Cfg::I8)
+                          acc = static_cast<uint32_t>(static_cast<int32_t>(acc) +
+                                                      static_cast<int32_t>(wv[i]));
+                        else
+                          acc = __float_as_uint(__fadd_rn(__uint_as_float(acc),
+                                                          __uint_as_float(wv[i])));
+                      }
+                    }
                   }
                 }
               }

@@ -42,6 +42,21 @@ __device__ __forceinline__ int quant_code(float v, float mult) {
   return max(-127, min(127, c));
 }
 
+// Low byte of the code rint(v * mult) for |v * mult| < 2^22: adding 1.5 * 2^23
+// moves the product into [2^23, 2^24), where the float spacing is 1, so the
+// addition itself rounds half-to-even to an integer held in the low mantissa
+// bits; the low byte is the two's-complement byte of that integer.  With
+// |v| <= amax and mult = fp32(127 / amax), |v * mult| <= 127 * (1 + 2^-24)^2,
+// which rounds to at most 127, so no clamp is needed (equal to quant_code).
+__device__ __forceinline__ uint32_t quant_byte_bits(float v, float mult) {
+  return __float_as_uint(__fadd_rn(__fmul_rn(v, mult), 12582912.0f));
+}
+// Pack the low bytes of four such patterns into one word (element 0 lowest).
+__device__ __forceinline__ uint32_t pack_code_bytes(uint32_t a, uint32_t b, uint32_t c,
+                                                    uint32_t d) {
+  return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
+}
+
 // Quantise `nseg` segments of `group` contiguous elements of the row-major
 // [rows, K] BF16 matrix x, each with its own symmetric scale.  TPR threads
 // cooperate on one segment, 16 elements per thread per step (two 128-bit
@@ -124,6 +139,147 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const __nv_bfloat16* __
       pk[j] = b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
     }
     *reinterpret_cast<uint4*>(q + base + c) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  }
+}
+
+// Persistent streaming variant.  A row group of TPR threads (1 or 2 warps)
+// owns CH chunks of 16 columns per thread, keeps the 1/s factors of those
+// columns in registers for its whole life, and streams its rows through a
+// ring of S shared-memory stages filled by 1-D bulk copies (one row per
+// stage), so the copy engine keeps S rows per group in flight while the
+// threads compute.  Per row: absmax pass and coding pass both read the row
+// from shared memory; codes leave in 128-bit stores.  Same arithmetic as
+// quant_rows_kernel.
+template <int TPR, int CH, int G, bool HAS_VEC>
+__global__ void __launch_bounds__(TPR * G) quant_stream_kernel(const __nv_bfloat16* __restrict__ x,
+                                                               const float* __restrict__ vec,
+                                                               int8_t* __restrict__ q,
+                                                               float* __restrict__ scales,
+                                                               int64_t nrows, int K, int S) {
+  constexpr int NW = TPR / 32;
+  extern __shared__ __align__(128) uint8_t qsm[];
+  const int g = threadIdx.x / TPR;            // row group within the block
+  const int t = threadIdx.x % TPR;
+  const int lane = threadIdx.x & 31;
+  const int wig = t >> 5;                     // warp within the group
+  const size_t row_bytes = static_cast<size_t>(K) * 2;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(qsm);                 // [G][S]
+  float* red = reinterpret_cast<float*>(qsm + G * S * 8);            // [G][NW]
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(qsm + G * S * 8 + G * NW * 4);
+  uint8_t* ring = qsm + 1024 + static_cast<size_t>(g) * S * row_bytes;
+  uint64_t* full = bars + g * S;
+
+  const int64_t group = static_cast<int64_t>(blockIdx.x) * G + g;
+  const int64_t ngroups = static_cast<int64_t>(gridDim.x) * G;
+  griddep_launch_dependents();  // a dependent GEMM may start its prologue
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < G * S; ++i) mbar_init(bars + i, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  // this thread's 1/s factors, kept in registers
+  float v[CH][16];
+#pragma unroll
+  for (int j = 0; j < CH; ++j) {
+    const int c = (j * TPR + t) * 16;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[j][i] = 1.0f;
+    if (HAS_VEC && c < K) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float4 s4 = __ldg(reinterpret_cast<const float4*>(vec + c) + i);
+        v[j][4 * i] = s4.x;
+        v[j][4 * i + 1] = s4.y;
+        v[j][4 * i + 2] = s4.z;
+        v[j][4 * i + 3] = s4.w;
+      }
+    }
+  }
+
+  // prologue: the first S rows of this group
+  int issued = 0;
+  if (t == 0) {
+    for (int i = 0; i < S; ++i) {
+      const int64_t r = group + static_cast<int64_t>(i) * ngroups;
+      if (r >= nrows) break;
+      mbar_arrive_expect_tx(full + i, static_cast<uint32_t>(row_bytes));
+      bulk_load(ring + i * row_bytes, x + r * K, static_cast<uint32_t>(row_bytes), full + i);
+      ++issued;
+    }
+  }
+  const int bar_id = 1 + g;
+  int stage = 0;
+  uint32_t phase = 0;
+  for (int64_t r = group, i = 0; r < nrows; r += ngroups, ++i) {
+    const bool ok = wait_bounded(full + stage, phase, abort_flag);
+    if (named_bar_or(bar_id, TPR, !ok)) break;
+    const uint8_t* row = ring + stage * row_bytes;
+    float amax = 0.0f;
+#pragma unroll
+    for (int j = 0; j < CH; ++j) {
+      const int c = (j * TPR + t) * 16;
+      if (c < K) {
+        float f[16];
+        bf16x8_to_f32(*reinterpret_cast<const uint4*>(row + 2 * c), *reinterpret_cast<float(*)[8]>(&f[0]));
+        bf16x8_to_f32(*reinterpret_cast<const uint4*>(row + 2 * c + 16), *reinterpret_cast<float(*)[8]>(&f[8]));
+#pragma unroll
+        for (int k = 0; k < 16; ++k) amax = fmaxf(amax, fabsf(HAS_VEC ? __fmul_rn(f[k], v[j][k]) : f[k]));
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    if (NW > 1) {
+      if (lane == 0) red[g * NW + wig] = amax;
+      named_bar_sync(bar_id, TPR);
+#pragma unroll
+      for (int w = 0; w < NW; ++w) amax = fmaxf(amax, red[g * NW + w]);
+    }
+    const float scale = __fdiv_rn(amax, 127.0f);
+    const float mult = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
+    if (t == 0) scales[r] = scale;
+    int8_t* qr = q + r * K;
+#pragma unroll
+    for (int j = 0; j < CH; ++j) {
+      const int c = (j * TPR + t) * 16;
+      if (c < K) {
+        float f[16];
+        bf16x8_to_f32(*reinterpret_cast<const uint4*>(row + 2 * c), *reinterpret_cast<float(*)[8]>(&f[0]));
+        bf16x8_to_f32(*reinterpret_cast<const uint4*>(row + 2 * c + 16), *reinterpret_cast<float(*)[8]>(&f[8]));
+        uint32_t pk[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          uint32_t b[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float xv = HAS_VEC ? __fmul_rn(f[4 * k + e], v[j][4 * k + e]) : f[4 * k + e];
+            b[e] = quant_byte_bits(xv, mult);
+          }
+          pk[k] = pack_code_bytes(b[0], b[1], b[2], b[3]);
+        }
+        *reinterpret_cast<uint4*>(qr + c) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
+    }
+    // every thread of the group is done with this stage (and with red[])
+    named_bar_sync(bar_id, TPR);
+    if (t == 0) {
+      const int64_t rn = r + static_cast<int64_t>(S) * ngroups;
+      if (rn < nrows) {
+        mbar_arrive_expect_tx(full + stage, static_cast<uint32_t>(row_bytes));
+        bulk_load(ring + stage * row_bytes, x + rn * K, static_cast<uint32_t>(row_bytes), full + stage);
+        ++issued;
+      }
+    }
+    if (++stage == S) { stage = 0; phase ^= 1u; }
+  }
+  // no copy may still be writing shared memory when the block exits
+  if (t == 0) {
+    for (int st = 0; st < S; ++st) {
+      const int n = issued / S + (st < issued % S ? 1 : 0);
+      if (n > 0) wait_drain(full + st, static_cast<uint32_t>((n - 1) & 1));
+    }
   }
 }
 

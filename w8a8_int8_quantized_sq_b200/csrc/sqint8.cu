@@ -42,7 +42,8 @@ EncodeTiledFn encode_fn() {
 // K-major 2-D operand: rows of `inner` elements, box of box_inner x box_rows,
 // 128-byte swizzle, out-of-bounds rows read as zero.
 bool make_map(CUtensorMap* m, const void* ptr, bool bf16, uint64_t inner, uint64_t rows,
-              uint32_t box_inner, uint32_t box_rows) {
+              uint32_t box_inner, uint32_t box_rows,
+              CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const uint64_t esz = bf16 ? 2 : 1;
@@ -52,7 +53,7 @@ bool make_map(CUtensorMap* m, const void* ptr, bool bf16, uint64_t inner, uint64
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
                    const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -85,7 +86,7 @@ sq_status launch_status() {
 }
 
 // ---------------------------------------------------------------- planning
-enum GemmKind { GK_I8_SCALE = 0, GK_I8_I32 = 1, GK_GS128 = 2, GK_BF16 = 3 };
+enum GemmKind { GK_I8_SCALE = 0, GK_I8_I32 = 1, GK_GS128 = 2, GK_BF16 = 3, GK_W8A16_CONV = 4 };
 
 struct GemmPlan {
   bool swap;
@@ -100,7 +101,7 @@ struct GemmPlan {
 
 GemmPlan plan_gemm(GemmKind kind, int64_t M, int64_t N, int64_t K, int sms) {
   GemmPlan p{};
-  const bool i8 = kind != GK_BF16;
+  const bool i8 = kind != GK_BF16 && kind != GK_W8A16_CONV;
   p.kb_total = static_cast<int>(K / (i8 ? 128 : 64));
   if (kind != GK_GS128 && M <= 32) {
     p.swap = true;
@@ -109,7 +110,16 @@ GemmPlan plan_gemm(GemmKind kind, int64_t M, int64_t N, int64_t K, int sms) {
     p.tiles_c = 1;
     p.stream_k = true;
     p.total_iters = static_cast<long long>(p.tiles_r) * p.kb_total;
-    p.grid = static_cast<int>(p.total_iters < sms ? p.total_iters : sms);
+    const int whole = p.tiles_r <= sms ? sms / p.tiles_r : 0;
+    if (whole > 0 && p.kb_total / whole <= 24) {
+      // short K ranges: whole splits, so every CTA owns one contiguous K range
+      // of one tile and runs a single epilogue (stream-K ranges with
+      // G = tiles * splits); long ranges use every SM instead
+      const int splits = whole > p.kb_total ? p.kb_total : whole;
+      p.grid = p.tiles_r * splits;
+    } else {
+      p.grid = sms;
+    }
     p.ws_bytes = kCounterBytes + static_cast<size_t>(p.grid) * 2 * 128 * p.bn * 4;
   } else {
     p.swap = false;
@@ -127,20 +137,46 @@ GemmPlan plan_gemm(GemmKind kind, int64_t M, int64_t N, int64_t K, int sms) {
 
 template <class Cfg>
 sq_status launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& g, int grid,
-                      cudaStream_t st) {
+                      cudaStream_t st, bool pdl) {
   const int smem = Cfg::smem_bytes(g.kb_total);
   if (smem > 232448) return SQ_ERR_SHAPE;
-  if (cudaFuncSetAttribute(gemm_kernel<Cfg>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-      cudaSuccess)
-    return SQ_ERR_CUDA;
-  gemm_kernel<Cfg><<<grid, Cfg::THREADS, smem, st>>>(a, b, g);
+  // Raise the kernel's dynamic shared-memory limit once per device (and only
+  // upwards), so steady-state launches make no attribute call.
+  static std::atomic<int> smem_set[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SQ_ERR_CUDA;
+  if (smem_set[dev].load(std::memory_order_acquire) < smem) {
+    if (cudaFuncSetAttribute(gemm_kernel<Cfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem) != cudaSuccess)
+      return SQ_ERR_CUDA;
+    int cur = smem_set[dev].load();
+    while (cur < smem && !smem_set[dev].compare_exchange_weak(cur, smem)) {
+    }
+  }
+  if (!pdl) {
+    gemm_kernel<Cfg><<<grid, Cfg::THREADS, smem, st>>>(a, b, g);
+    return launch_status();
+  }
+  // programmatic dependent launch: the kernel may start while the preceding
+  // kernel on the stream runs; it requests only weights before griddep_wait
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(Cfg::THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, gemm_kernel<Cfg>, a, b, g) != cudaSuccess) return SQ_ERR_CUDA;
   return launch_status();
 }
 
 // act: q_a int8 [M,K] or x bf16 [M,K]; wt: q_w int8 [N,K] or bf16 [N,K].
 sq_status run_gemm(GemmKind kind, const void* act, const void* wt, const float* s_tok,
                    const float* s_ch, const float* s_blk, void* out, int64_t M, int64_t N,
-                   int64_t K, void* ws, size_t ws_bytes, cudaStream_t st) {
+                   int64_t K, void* ws, size_t ws_bytes, cudaStream_t st, bool pdl = false) {
   const int sms = num_sms();
   if (sms <= 0) return SQ_ERR_CUDA;
   const GemmPlan p = plan_gemm(kind, M, N, K, sms);
@@ -148,14 +184,22 @@ sq_status run_gemm(GemmKind kind, const void* act, const void* wt, const float* 
     return SQ_ERR_SHAPE;
   if (p.ws_bytes > 0 && (!ws || ws_bytes < p.ws_bytes)) return SQ_ERR_WORKSPACE;
   if (ws && !aligned16(ws)) return SQ_ERR_ALIGN;
-  const bool bf16 = kind == GK_BF16;
+  const bool conv = kind == GK_W8A16_CONV;
+  const bool bf16 = kind == GK_BF16 || conv;
   const uint32_t kbe = bf16 ? 64 : 128;
   CUtensorMap ta, tb;
   const void* a_ptr = p.swap ? wt : act;
   const void* b_ptr = p.swap ? act : wt;
   const uint64_t a_rows = static_cast<uint64_t>(p.swap ? N : M);
   const uint64_t b_rows = static_cast<uint64_t>(p.swap ? M : N);
-  if (!make_map(&ta, a_ptr, bf16, static_cast<uint64_t>(K), a_rows, kbe, 128)) return SQ_ERR_CUDA;
+  if (conv) {
+    if (!p.swap) return SQ_ERR_SHAPE;
+    // raw int8 weight rows, 128 bytes (two 64-element K blocks) per row per box
+    if (!make_map(&ta, a_ptr, false, static_cast<uint64_t>(K), a_rows, 128, 128))
+      return SQ_ERR_CUDA;
+  } else if (!make_map(&ta, a_ptr, bf16, static_cast<uint64_t>(K), a_rows, kbe, 128)) {
+    return SQ_ERR_CUDA;
+  }
   if (!make_map(&tb, b_ptr, bf16, static_cast<uint64_t>(K), b_rows, kbe, p.bn)) return SQ_ERR_CUDA;
 
   GemmArgs g{};
@@ -180,30 +224,41 @@ sq_status run_gemm(GemmKind kind, const void* act, const void* wt, const float* 
   switch (kind) {
     case GK_I8_SCALE:
       if (p.swap && p.bn == 16)
-        return launch_gemm<GemmCfg<true, 16, 8, true, EPI_SCALE>>(ta, tb, g, p.grid, st);
+        return launch_gemm<GemmCfg<true, 16, 8, true, EPI_SCALE>>(ta, tb, g, p.grid, st, pdl);
       if (p.swap)
-        return launch_gemm<GemmCfg<true, 32, 8, true, EPI_SCALE>>(ta, tb, g, p.grid, st);
-      return launch_gemm<GemmCfg<true, 256, 4, false, EPI_SCALE>>(ta, tb, g, p.grid, st);
+        return launch_gemm<GemmCfg<true, 32, 8, true, EPI_SCALE>>(ta, tb, g, p.grid, st, pdl);
+      return launch_gemm<GemmCfg<true, 256, 4, false, EPI_SCALE>>(ta, tb, g, p.grid, st, pdl);
     case GK_I8_I32:
       if (p.swap && p.bn == 16)
-        return launch_gemm<GemmCfg<true, 16, 8, true, EPI_I32>>(ta, tb, g, p.grid, st);
+        return launch_gemm<GemmCfg<true, 16, 8, true, EPI_I32>>(ta, tb, g, p.grid, st, pdl);
       if (p.swap)
-        return launch_gemm<GemmCfg<true, 32, 8, true, EPI_I32>>(ta, tb, g, p.grid, st);
-      return launch_gemm<GemmCfg<true, 256, 4, false, EPI_I32>>(ta, tb, g, p.grid, st);
+        return launch_gemm<GemmCfg<true, 32, 8, true, EPI_I32>>(ta, tb, g, p.grid, st, pdl);
+      return launch_gemm<GemmCfg<true, 256, 4, false, EPI_I32>>(ta, tb, g, p.grid, st, pdl);
     case GK_GS128:
-      return launch_gemm<GemmCfg<true, 128, 4, false, EPI_GS128>>(ta, tb, g, p.grid, st);
+      return launch_gemm<GemmCfg<true, 128, 4, false, EPI_GS128>>(ta, tb, g, p.grid, st, pdl);
     case GK_BF16:
       if (p.swap && p.bn == 16)
-        return launch_gemm<GemmCfg<false, 16, 8, true, EPI_SCALE>>(ta, tb, g, p.grid, st);
+        return launch_gemm<GemmCfg<false, 16, 8, true, EPI_SCALE>>(ta, tb, g, p.grid, st, pdl);
       if (p.swap)
-        return launch_gemm<GemmCfg<false, 32, 8, true, EPI_SCALE>>(ta, tb, g, p.grid, st);
-      return launch_gemm<GemmCfg<false, 256, 4, false, EPI_SCALE>>(ta, tb, g, p.grid, st);
+        return launch_gemm<GemmCfg<false, 32, 8, true, EPI_SCALE>>(ta, tb, g, p.grid, st, pdl);
+      return launch_gemm<GemmCfg<false, 256, 4, false, EPI_SCALE>>(ta, tb, g, p.grid, st, pdl);
+    case GK_W8A16_CONV:
+      if (p.bn == 16)
+        return launch_gemm<GemmCfg<false, 16, 12, true, EPI_SCALE, true, 5>>(ta, tb, g, p.grid,
+                                                                            st, pdl);
+      return launch_gemm<GemmCfg<false, 32, 8, true, EPI_SCALE, true, 5>>(ta, tb, g, p.grid, st,
+                                                                         pdl);
   }
   return SQ_ERR_SHAPE;
 }
 
-// W8A16 workspace: [counter region][stream-K slots][bf16 weights N x K]
+// W8A16 workspace.  M <= 32 (dequant on load): [counter region][stream-K
+// slots].  Larger M: [counter region][bf16 weights N x K].
 size_t w8a16_ws_bytes(int64_t M, int64_t N, int64_t K, int sms, size_t* w_off) {
+  if (M <= 32) {
+    if (w_off) *w_off = 0;
+    return plan_gemm(GK_W8A16_CONV, M, N, K, sms).ws_bytes;
+  }
   const GemmPlan p = plan_gemm(GK_BF16, M, N, K, sms);
   const size_t off = align256(p.ws_bytes > kCounterBytes ? p.ws_bytes : kCounterBytes);
   if (w_off) *w_off = off;
@@ -222,9 +277,66 @@ sq_status launch_quant(const void* x, const float* vec, int8_t* q, float* scales
   return launch_status();
 }
 
+template <int TPR, int CH, int G>
+sq_status launch_quant_stream(const void* x, const float* vec, int8_t* q, float* scales,
+                              int64_t rows, int64_t K, cudaStream_t st) {
+  const size_t row_bytes = static_cast<size_t>(K) * 2;
+  // ring depth: about 100 KB of rows per block (two blocks per SM), at least
+  // two rows per group so one is in flight while the other is processed
+  int S = static_cast<int>((100u << 10) / (G * row_bytes));
+  S = S < 2 ? 2 : (S > 8 ? 8 : S);
+  const size_t smem = 1024 + static_cast<size_t>(G) * S * row_bytes;
+  if (smem > 232448) return SQ_ERR_SHAPE;
+  const int sms = num_sms();
+  if (sms <= 0) return SQ_ERR_CUDA;
+  int64_t blocks = (rows + G - 1) / G;
+  if (blocks > 2 * sms) blocks = 2 * sms;
+  auto kern = vec ? quant_stream_kernel<TPR, CH, G, true> : quant_stream_kernel<TPR, CH, G, false>;
+  static std::atomic<int> smem_set[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SQ_ERR_CUDA;
+  const int flag = vec ? 2 : 1;
+  if ((smem_set[dev].load() & flag) == 0) {
+    if (cudaFuncSetAttribute(quant_stream_kernel<TPR, CH, G, true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, 232448) != cudaSuccess ||
+        cudaFuncSetAttribute(quant_stream_kernel<TPR, CH, G, false>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, 232448) != cudaSuccess)
+      return SQ_ERR_CUDA;
+    smem_set[dev].fetch_or(3);
+  }
+  kern<<<static_cast<unsigned>(blocks), TPR * G, smem, st>>>(
+      static_cast<const __nv_bfloat16*>(x), vec, q, scales, rows, static_cast<int>(K), S);
+  return launch_status();
+}
+
+template <int TPR, int G>
+sq_status launch_quant_stream_ch(int ch, const void* x, const float* vec, int8_t* q,
+                                 float* scales, int64_t rows, int64_t K, cudaStream_t st) {
+  switch (ch) {
+    case 1: return launch_quant_stream<TPR, 1, G>(x, vec, q, scales, rows, K, st);
+    case 2: return launch_quant_stream<TPR, 2, G>(x, vec, q, scales, rows, K, st);
+    case 3: return launch_quant_stream<TPR, 3, G>(x, vec, q, scales, rows, K, st);
+    case 4: return launch_quant_stream<TPR, 4, G>(x, vec, q, scales, rows, K, st);
+    case 5: return launch_quant_stream<TPR, 5, G>(x, vec, q, scales, rows, K, st);
+    default: return launch_quant_stream<TPR, 6, G>(x, vec, q, scales, rows, K, st);
+  }
+}
+
+// One scale per row of K elements (K <= 24576): the streaming kernel with the
+// fewest threads per row that keeps at most 6 chunks of 16 columns (and
+// their 1/s factors) per thread.
+sq_status quant_per_row(const void* x, const float* vec, int8_t* q, float* scales, int64_t rows,
+                        int64_t K, cudaStream_t st) {
+  const int64_t c64 = (K + 1023) / 1024, c128 = (K + 2047) / 2048, c256 = (K + 4095) / 4096;
+  if (c64 <= 6) return launch_quant_stream_ch<64, 4>(static_cast<int>(c64), x, vec, q, scales, rows, K, st);
+  if (c128 <= 6) return launch_quant_stream_ch<128, 1>(static_cast<int>(c128), x, vec, q, scales, rows, K, st);
+  return launch_quant_stream_ch<256, 1>(static_cast<int>(c256), x, vec, q, scales, rows, K, st);
+}
+
 sq_status quant_rows(const void* x, const float* vec, int8_t* q, float* scales, int64_t nseg,
                      int64_t K, int64_t group, cudaStream_t st) {
   if (nseg == 0) return SQ_OK;
+  if (group == K && K <= 256 * 16 * 6) return quant_per_row(x, vec, q, scales, nseg, K, st);
   if (group == 128) {
     return vec ? launch_quant<8, true>(x, vec, q, scales, nseg, K, group, st)
                : launch_quant<8, false>(x, vec, q, scales, nseg, K, group, st);
@@ -330,6 +442,27 @@ sq_status w8a8_scaled_mm(const int8_t* q_a, const float* s_tok, const int8_t* q_
                   ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
+sq_status sq_w8a8_linear(const void* x_bf16, const float* inv_smooth, const int8_t* q_w,
+                         const float* s_ch, void* y_bf16, int8_t* q_a, float* s_tok, int64_t M,
+                         int64_t N, int64_t K, void* workspace, size_t ws_bytes, void* stream) {
+  sq_status s = check_mnk(M, N, K);
+  if (s != SQ_OK) return s;
+  if (M == 0) return SQ_OK;
+  if (!x_bf16 || !q_w || !s_ch || !y_bf16 || !q_a || !s_tok) return SQ_ERR_NULL;
+  if (!aligned16(x_bf16) || !aligned16(q_w) || !aligned16(s_ch) || !aligned16(y_bf16) ||
+      !aligned16(q_a) || !aligned16(s_tok) || (inv_smooth && !aligned16(inv_smooth)))
+    return SQ_ERR_ALIGN;
+  const int sms = num_sms();
+  if (sms <= 0) return SQ_ERR_CUDA;
+  const GemmPlan p = plan_gemm(GK_I8_SCALE, M, N, K, sms);
+  if (p.ws_bytes > 0 && (!workspace || ws_bytes < p.ws_bytes)) return SQ_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  s = quant_rows(x_bf16, inv_smooth, q_a, s_tok, M, K, K, st);
+  if (s != SQ_OK) return s;
+  return run_gemm(GK_I8_SCALE, q_a, q_w, s_tok, s_ch, nullptr, y_bf16, M, N, K, workspace,
+                  ws_bytes, st, /*pdl=*/true);
+}
+
 sq_status w8a8_mm_i32(const int8_t* q_a, const int8_t* q_w, int32_t* acc, int64_t M, int64_t N,
                       int64_t K, void* workspace, size_t ws_bytes, void* stream) {
   sq_status s = check_mnk(M, N, K);
@@ -371,6 +504,9 @@ sq_status w8a16_mm(const void* x_bf16, const int8_t* q_w, const float* s_ch, voi
   if (!workspace || ws_bytes < need) return SQ_ERR_WORKSPACE;
   if (!aligned16(workspace)) return SQ_ERR_ALIGN;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (M <= 32)  // weight-read bound: int8 weights are converted on load, in the GEMM
+    return run_gemm(GK_W8A16_CONV, x_bf16, q_w, nullptr, s_ch, nullptr, y_bf16, M, N, K,
+                    workspace, ws_bytes, st);
   __nv_bfloat16* wb = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(workspace) + w_off);
   const int64_t n16 = N * K / 16;
   const int64_t blocks = (n16 + 255) / 256 < 4 * sms ? (n16 + 255) / 256 : 4 * sms;
