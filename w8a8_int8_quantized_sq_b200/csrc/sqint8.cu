@@ -2,10 +2,12 @@
 // argument checks, launch planning, tensor-map encoding and kernel launches.
 // The library holds no device memory of its own except one error word.
 #include <atomic>
+#include <cstdlib>
 #include <mutex>
 
 #include "../../include/sqint8.h"
 #include "gemm.cuh"
+#include "gemm2.cuh"
 #include "quant.cuh"
 
 using namespace sq;
@@ -89,6 +91,7 @@ sq_status launch_status() {
 enum GemmKind { GK_I8_SCALE = 0, GK_I8_I32 = 1, GK_GS128 = 2, GK_BF16 = 3, GK_W8A16_CONV = 4 };
 
 struct GemmPlan {
+  bool pair;  // CTA-pair kernel (256 x 256 tiles per cluster of two)
   bool swap;
   int bn;
   bool stream_k;
@@ -98,6 +101,17 @@ struct GemmPlan {
   long long total_iters;
   size_t ws_bytes;  // counter region + stream-K slots (0: no workspace)
 };
+
+// The CTA-pair kernel serves the large-token W8A8 shapes unless the
+// environment variable SQ_GEMM_PAIR is set to 0 (then one CTA per 128 x 256
+// tile is used, e.g. for comparisons).
+bool pair_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("SQ_GEMM_PAIR");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
 
 GemmPlan plan_gemm(GemmKind kind, int64_t M, int64_t N, int64_t K, int sms) {
   GemmPlan p{};
@@ -121,6 +135,16 @@ GemmPlan plan_gemm(GemmKind kind, int64_t M, int64_t N, int64_t K, int sms) {
       p.grid = sms;
     }
     p.ws_bytes = kCounterBytes + static_cast<size_t>(p.grid) * 2 * 128 * p.bn * 4;
+  } else if ((kind == GK_I8_SCALE || kind == GK_I8_I32) && pair_enabled()) {
+    p.pair = true;
+    p.swap = false;
+    p.bn = 256;
+    p.tiles_r = static_cast<int>((M + 255) / 256);
+    p.tiles_c = static_cast<int>((N + 255) / 256);
+    p.stream_k = false;
+    p.total_iters = static_cast<long long>(p.tiles_r) * p.tiles_c * p.kb_total;
+    p.grid = 0;  // decided at launch from the active-cluster limit
+    p.ws_bytes = 0;
   } else {
     p.swap = false;
     p.bn = kind == GK_GS128 ? 128 : 256;
@@ -173,6 +197,42 @@ sq_status launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const GemmArgs
   return launch_status();
 }
 
+template <class Cfg>
+sq_status launch_gemm2(const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& g,
+                       cudaStream_t st, bool pdl) {
+  const int smem = Cfg::smem_bytes();
+  static std::atomic<int> max_clusters[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SQ_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(Cfg::THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 2 : 1;
+  int mc = max_clusters[dev].load(std::memory_order_acquire);
+  if (mc <= 0) {
+    if (cudaFuncSetAttribute(gemm2_kernel<Cfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem) != cudaSuccess)
+      return SQ_ERR_CUDA;
+    cfg.gridDim = dim3(2);
+    if (cudaOccupancyMaxActiveClusters(&mc, gemm2_kernel<Cfg>, &cfg) != cudaSuccess || mc <= 0)
+      return SQ_ERR_CUDA;
+    max_clusters[dev].store(mc, std::memory_order_release);
+  }
+  const int clusters = g.num_tiles < mc ? g.num_tiles : mc;
+  cfg.gridDim = dim3(2 * clusters);
+  if (cudaLaunchKernelEx(&cfg, gemm2_kernel<Cfg>, a, b, g) != cudaSuccess) return SQ_ERR_CUDA;
+  return launch_status();
+}
+
 // act: q_a int8 [M,K] or x bf16 [M,K]; wt: q_w int8 [N,K] or bf16 [N,K].
 sq_status run_gemm(GemmKind kind, const void* act, const void* wt, const float* s_tok,
                    const float* s_ch, const float* s_blk, void* out, int64_t M, int64_t N,
@@ -200,7 +260,9 @@ sq_status run_gemm(GemmKind kind, const void* act, const void* wt, const float* 
   } else if (!make_map(&ta, a_ptr, bf16, static_cast<uint64_t>(K), a_rows, kbe, 128)) {
     return SQ_ERR_CUDA;
   }
-  if (!make_map(&tb, b_ptr, bf16, static_cast<uint64_t>(K), b_rows, kbe, p.bn)) return SQ_ERR_CUDA;
+  // the pair kernel stages 128 of the tile's 256 weight rows in each CTA
+  if (!make_map(&tb, b_ptr, bf16, static_cast<uint64_t>(K), b_rows, kbe, p.pair ? 128 : p.bn))
+    return SQ_ERR_CUDA;
 
   GemmArgs g{};
   g.R = static_cast<int>(p.swap ? N : M);
@@ -221,6 +283,10 @@ sq_status run_gemm(GemmKind kind, const void* act, const void* wt, const float* 
   g.ws = p.ws_bytes ? reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + kCounterBytes)
                     : nullptr;
 
+  if (p.pair) {
+    if (kind == GK_I8_SCALE) return launch_gemm2<Gemm2Cfg<EPI_SCALE, 6>>(ta, tb, g, st, pdl);
+    return launch_gemm2<Gemm2Cfg<EPI_I32, 6>>(ta, tb, g, st, pdl);
+  }
   switch (kind) {
     case GK_I8_SCALE:
       if (p.swap && p.bn == 16)
