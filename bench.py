@@ -36,6 +36,20 @@ INT8_PER_BF16 = 2.0          # dense INT8 ops per dense BF16 flop (4.5 / 2.25 PF
 INT8_NOMINAL_TOPS = 4500.0   # dense INT8, nominal B200
 
 
+def gemm_traffic():
+    """DRAM bytes per launch of the prefill GEMM from the committed ncu record,
+    or None if the kernel sources changed since it was captured."""
+    import hashlib
+    try:
+        rec = json.load(open(os.path.join(ROOT, "profiles", "gemm2_w8a8_prefill_traffic.json")))
+        h = hashlib.sha256()
+        for src in rec["sources"]:
+            h.update(open(os.path.join(ROOT, src), "rb").read())
+        return rec["traffic_bytes_per_launch"] if h.hexdigest() == rec["sources_sha256"] else None
+    except Exception:
+        return None
+
+
 def load_peaks():
     try:
         d = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
@@ -350,11 +364,13 @@ def main():
                    "l2": "inputs larger than L2 (q_w 178 MB, x 84 MB, y 570 MB)",
                    "step": "sq_quant_per_token + w8a8_scaled_mm"},
         "pct_of_int8_nominal": 100.0 * value / world / INT8_NOMINAL_TOPS,
-        "roofline": {"bound": "tensor", "kernel": "gemm_kernel (W8A8, 128x256 tiles)",
+        "roofline": {"bound": "tensor", "kernel": "gemm2_kernel (W8A8, CTA pairs, 256x256 tiles)",
                      "achieved": gemm_tops, "peak": int8_peak, "unit": "TOPS",
                      "frac": gemm_tops / int8_peak,
                      "peak_source": f"{peaks['source']} bf16 burst x {INT8_PER_BF16:g}",
-                     "traffic": None},
+                     "frac_of_sustained": gemm_tops / (peaks["bf16_tflops_sustained"] * INT8_PER_BF16),
+                     "traffic": gemm_traffic(),
+                     "algorithmic_bytes": algo_bytes_w8a8(M, N, K)},
         "split_ms": {"quant": quant_s * 1e3, "gemm": gemm_s * 1e3},
         "quant_hbm": {"achieved_gbs": algo_bytes_quant(M, K) / quant_s / 1e9,
                       "peak_gbs": peaks["hbm_gbs"],
