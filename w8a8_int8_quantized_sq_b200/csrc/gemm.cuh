@@ -167,9 +167,10 @@ struct SegIter {
 // --------------------------------------------------------------- epilogue
 // Scale/convert/store CW accumulator columns [c0, c0 + CW) of MMA row rr of
 // tile (rt, ct).  v holds int32 (I8) or fp32 bits (BF16) accumulators.
+// policy != 0: the 16-byte BF16 output stores carry that L2 eviction hint.
 template <class Cfg>
 __device__ __forceinline__ void store_chunk(const GemmArgs& g, int rt, int ct, int rr, int c0,
-                                            const uint32_t (&v)[Cfg::CW]) {
+                                            const uint32_t (&v)[Cfg::CW], uint64_t policy = 0) {
   constexpr int CW = Cfg::CW;
   const int r = rt * Cfg::BM + rr;
   const int cb = ct * Cfg::BN + c0;
@@ -203,9 +204,10 @@ __device__ __forceinline__ void store_chunk(const GemmArgs& g, int rt, int ct, i
             f[i] = __fmul_rn(__uint_as_float(v[j + i]), sc[i]);
           }
         }
-        *reinterpret_cast<uint4*>(out + n) =
-            make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
-                       pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+        const uint4 o = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                                   pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+        if (policy) st_global_v4_hint(out + n, o, policy);
+        else *reinterpret_cast<uint4*>(out + n) = o;
       }
     }
   } else {

@@ -21,16 +21,19 @@
 
 namespace sq {
 
-template <int EPI_, int STAGES_>
+// I8_ = true: W8A8 (kind::i8, int32 accumulators); false: BF16 operands
+// (kind::f16, fp32 accumulators), the large-token W8A16 shape after the
+// exact int8 -> bf16 weight conversion.
+template <int EPI_, int STAGES_, bool I8_ = true>
 struct Gemm2Cfg {
-  static constexpr bool I8 = true;
+  static constexpr bool I8 = I8_;
   static constexpr bool SWAP = false;
   static constexpr int EPI = EPI_;
   static constexpr int STAGES = STAGES_;
   static constexpr int BM = 128;        // token rows per CTA (256 per pair)
   static constexpr int BN = 256;        // output columns per pair tile
   static constexpr int BN_CTA = 128;    // weight rows staged by each CTA
-  static constexpr int KB_ELEMS = 128;  // int8 K elements per stage
+  static constexpr int KB_ELEMS = I8 ? 128 : 64;  // K elements per 128-byte stage row
   static constexpr int A_BYTES = BM * 128;
   static constexpr int B_BYTES = BN_CTA * 128;
   static constexpr int NE = 4;
@@ -101,6 +104,10 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       tma_prefetch_desc(&tmA);
       tma_prefetch_desc(&tmB);
       const uint32_t full_leader = mapa_shared(smem_u32(full), 0);
+      // activations are re-read by every weight column tile: keep them in L2
+      const uint64_t pol_act = policy_evict_last();
+      // a weight tile is read by the concurrent clusters of its column, then not again
+      const uint64_t pol_wt = policy_evict_normal();
       uint32_t stage = 0, phase = 0;
       long long fills = 0;
       bool ok = true;
@@ -110,7 +117,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       int pend_kb[STAGES], pend_row[STAGES];
       auto act_load = [&](int st, int kb, int row) {
         tma_load_2d_pair(smA + st * Cfg::A_BYTES, &tmA, kb * Cfg::KB_ELEMS, row,
-                         full_leader + st * 8);
+                         full_leader + st * 8, pol_act);
       };
       auto release_pending = [&]() {
         griddep_wait();
@@ -130,7 +137,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           }
           if (leader) mbar_arrive_expect_tx(full + stage, 2 * (Cfg::A_BYTES + Cfg::B_BYTES));
           tma_load_2d_pair(smB + stage * Cfg::B_BYTES, &tmB, kb * Cfg::KB_ELEMS, b_row,
-                           full_leader + stage * 8);
+                           full_leader + stage * 8, pol_wt);
           if (waited) {
             act_load(stage, kb, a_row);
           } else {
@@ -156,7 +163,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   } else if (warp == 1) {
     // ----------------------------------------------- MMA issuer (leader)
     if (leader && lane == 0) {
-      const uint32_t idesc = idesc_i8_s32_m256(BN);
+      const uint32_t idesc = Cfg::I8 ? idesc_i8_s32_m256(BN) : idesc_bf16_f32_m256(BN);
       uint32_t stage = 0, phase = 0, local = 0;
       bool ok = true;
       for (int t = cluster; ok && t < g.num_tiles; t += nclusters, ++local) {
@@ -170,9 +177,14 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           const uint32_t sa = smem_u32(smA + stage * Cfg::A_BYTES);
           const uint32_t sb = smem_u32(smB + stage * Cfg::B_BYTES);
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            mma_i8_pair(d, smem_desc_sw128(sa + k * 32), smem_desc_sw128(sb + k * 32), idesc,
-                        (kb > 0 || k > 0) ? 1u : 0u);
+          for (int k = 0; k < 4; ++k) {
+            if constexpr (Cfg::I8)
+              mma_i8_pair(d, smem_desc_sw128(sa + k * 32), smem_desc_sw128(sb + k * 32), idesc,
+                          (kb > 0 || k > 0) ? 1u : 0u);
+            else
+              mma_bf16_pair(d, smem_desc_sw128(sa + k * 32), smem_desc_sw128(sb + k * 32), idesc,
+                            (kb > 0 || k > 0) ? 1u : 0u);
+          }
           mma_commit_pair_both(empty + stage);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
@@ -186,6 +198,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     griddep_wait();
+    const uint64_t pol_out = policy_evict_first();  // the output is not re-read here
     const int q = warp & 3;
     const int rr = q * 32 + lane;
     const int nthr = NE * 32;
@@ -202,7 +215,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       for (int c = 0; c < BN; c += Cfg::CW) {
         uint32_t v[Cfg::CW];
         tmem_ld32(lane_base + a * BN + c, v);
-        store_chunk<Cfg>(g, rt128, ct, rr, c, v);
+        store_chunk<Cfg>(g, rt128, ct, rr, c, v, pol_out);
       }
       tc_fence_before();
       __syncwarp();

@@ -135,7 +135,7 @@ GemmPlan plan_gemm(GemmKind kind, int64_t M, int64_t N, int64_t K, int sms) {
       p.grid = sms;
     }
     p.ws_bytes = kCounterBytes + static_cast<size_t>(p.grid) * 2 * 128 * p.bn * 4;
-  } else if ((kind == GK_I8_SCALE || kind == GK_I8_I32) && pair_enabled()) {
+  } else if ((kind == GK_I8_SCALE || kind == GK_I8_I32 || kind == GK_BF16) && pair_enabled()) {
     p.pair = true;
     p.swap = false;
     p.bn = 256;
@@ -285,6 +285,8 @@ sq_status run_gemm(GemmKind kind, const void* act, const void* wt, const float* 
 
   if (p.pair) {
     if (kind == GK_I8_SCALE) return launch_gemm2<Gemm2Cfg<EPI_SCALE, 6>>(ta, tb, g, st, pdl);
+    if (kind == GK_BF16)
+      return launch_gemm2<Gemm2Cfg<EPI_SCALE, 6, false>>(ta, tb, g, st, pdl);
     return launch_gemm2<Gemm2Cfg<EPI_I32, 6>>(ta, tb, g, st, pdl);
   }
   switch (kind) {
