@@ -61,11 +61,13 @@ __host__ __device__ constexpr int pow2_at_least(int v) {
 // weight rows, RK K blocks per raw shared-memory stage (TMA, 128-byte
 // swizzle).  Eight converter warps expand a whole raw stage exactly to bf16
 // and write it straight into a ring of STAGES A tiles in tensor memory
-// (tcgen05.st; 32 columns of two bf16 per 128-lane row), then wait for their
-// stores once and release the raw stage; the MMA reads A from tensor memory.
-// A second producer thread loads each K block's B tile directly into a
-// shared-memory ring that shadows the A ring, so the raw ring can be deeper
-// than the A ring: the raw loads stay in flight while a stage is converted.  Keeping A out of shared
+// (tcgen05.st; 32 columns of two bf16 per 128-lane row per K block), then wait
+// for their stores once and release the raw stage; the MMA reads A from tensor
+// memory.  A second producer thread loads the K blocks' B tiles into their own
+// shared-memory ring.  Everything moves in groups of RK K blocks (one raw
+// stage, one A stage, one B stage): one hand-off and one tcgen05.commit per
+// 4 x RK MMAs, because short N = 16 MMAs committed one K block at a time keep
+// the tensor pipe waiting on each commit.  Keeping A out of shared
 // memory leaves 2 bytes of shared-memory traffic per weight byte instead of 6.
 template <bool I8_, int BN_, int STAGES_, bool SWAP_, int EPI_, bool CONV_ = false,
           int RSTAGES_ = 0>
@@ -98,17 +100,23 @@ struct GemmCfg {
   static constexpr int NSUB = (SWAP && EPI != EPI_GS128) ? 4 : 1;
   static constexpr int ACC_COLS = NACC * NSUB * BN;
   static constexpr int A_TMEM_COLS = 32;  // one 128 x 64 bf16 A tile in tensor memory
+  // CONV: an A stage holds the RK converted K blocks of one raw stage
   static constexpr int TMEM_COLS = CONV ? 512 : pow2_at_least(ACC_COLS);
   static constexpr int CW = BN < 32 ? BN : 32;  // columns per tcgen05.ld
   static constexpr int CPT = BN / (NE / 4);     // columns owned by one epilogue thread
   static constexpr int SBLK_STRIDE = BN + 4;    // floats per K block in the staged s_blk
   // shared memory carve-up (offsets from a 1024-byte aligned base)
   static constexpr int A_SMEM_BYTES = CONV ? 0 : A_BYTES;  // CONV: A lives in TMEM
+  // CONV: the B tiles have their own ring of stages of RK tiles (64 KB), so
+  // their loads run ahead of the MMAs instead of following the A stages
+  static constexpr int BSTAGES = CONV ? (65536 / (RK * B_BYTES)) : STAGES;
+  static constexpr int B_RING_BYTES = CONV ? BSTAGES * RK * B_BYTES : STAGES * B_BYTES;
   static constexpr int OFF_RAW = 0;
   static constexpr int OFF_A = OFF_RAW + RSTAGES * RAW_BYTES;
   static constexpr int OFF_B = OFF_A + STAGES * A_SMEM_BYTES;
-  static constexpr int OFF_BAR = OFF_B + STAGES * B_BYTES;
-  static constexpr int NUM_BARS = 2 * STAGES + 2 * NACC + 1 + 2 * RSTAGES;
+  static constexpr int OFF_BAR = OFF_B + B_RING_BYTES;
+  static constexpr int NUM_BARS =
+      2 * STAGES + 2 * NACC + 1 + 2 * RSTAGES + (CONV ? 2 * BSTAGES : 0);
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int OFF_SBLK = (OFF_MISC + 16 + 15) / 16 * 16;
   static constexpr int smem_bytes(int kb_total) {
@@ -118,7 +126,7 @@ struct GemmCfg {
   static_assert(EPI != EPI_GS128 || (I8 && !SWAP && BN % 64 == 0), "gs128 layout");
   static_assert(!CONV || (!I8 && SWAP && EPI == EPI_SCALE), "dequant-on-load is W8A16, swapped");
   static_assert(!CONV || (RAW_BYTES % 1024 == 0 && B_BYTES % 16 == 0), "raw stage alignment");
-  static_assert(!CONV || ACC_COLS + STAGES * A_TMEM_COLS <= 512, "tensor memory A ring");
+  static_assert(!CONV || ACC_COLS + STAGES * RK * A_TMEM_COLS <= 512, "tensor memory A ring");
 
   static_assert(TMEM_COLS <= 512, "tensor memory");
 };
@@ -286,6 +294,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   uint64_t* drain = tempty + NACC;
   uint64_t* raw_full = drain + 1;             // CONV: producer -> converters
   uint64_t* raw_empty = raw_full + Cfg::RSTAGES;  // CONV: converters -> producer
+  uint64_t* b_full = raw_empty + Cfg::RSTAGES;    // CONV: B producer -> MMA
+  uint64_t* b_empty = b_full + Cfg::BSTAGES;      // CONV: MMA -> B producer
   uint8_t* smRaw = smem + Cfg::OFF_RAW;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::OFF_MISC + 4);
@@ -306,13 +316,15 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     }
     mbar_init(drain, 1);
     if constexpr (Cfg::CONV) {
-      // the converted stage completes on the converter warps' arrivals plus
-      // the B tile's transaction bytes
-      // converted stage: converter warps' arrivals + the producer's B tile
-      for (int s = 0; s < STAGES; ++s) mbar_init(full + s, Cfg::NCV + 1);
+      // a converted A stage completes on the converter warps' arrivals
+      for (int s = 0; s < STAGES; ++s) mbar_init(full + s, Cfg::NCV);
       for (int s = 0; s < Cfg::RSTAGES; ++s) {
         mbar_init(raw_full + s, 1);
         mbar_init(raw_empty + s, Cfg::NCV);
+      }
+      for (int s = 0; s < Cfg::BSTAGES; ++s) {
+        mbar_init(b_full + s, 1);
+        mbar_init(b_empty + s, 1);
       }
     }
     *abort_flag = 0;
@@ -370,17 +382,20 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       bool ok = true;
       while (ok && it.next(g, s)) {
         const int ct = s.tile / g.tiles_r;
-        for (int kb = s.kb0; kb < s.kb1; ++kb) {
-          if (!wait_bounded(empty + cs, cph ^ 1u, abort_flag)) { ok = false; break; }
-          mbar_arrive_expect_tx(full + cs, Cfg::B_BYTES);
-          tma_load_2d(smB + cs * Cfg::B_BYTES, &tmB, kb * Cfg::KB_ELEMS, ct * BN, full + cs);
+        for (int kb = s.kb0; kb < s.kb1; kb += Cfg::RK) {
+          const int n = s.kb1 - kb < Cfg::RK ? s.kb1 - kb : Cfg::RK;
+          if (!wait_bounded(b_empty + cs, cph ^ 1u, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(b_full + cs, n * Cfg::B_BYTES);
+          for (int c = 0; c < n; ++c)
+            tma_load_2d(smB + (cs * Cfg::RK + c) * Cfg::B_BYTES, &tmB, (kb + c) * Cfg::KB_ELEMS,
+                        ct * BN, b_full + cs);
           ++bfills;
-          if (++cs == STAGES) { cs = 0; cph ^= 1u; }
+          if (++cs == Cfg::BSTAGES) { cs = 0; cph ^= 1u; }
         }
       }
-      for (int st = 0; st < STAGES; ++st) {
-        const long long n = bfills / STAGES + (st < bfills % STAGES ? 1 : 0);
-        if (n > 0) wait_drain(full + st, static_cast<uint32_t>((n - 1) & 1));
+      for (int st = 0; st < Cfg::BSTAGES; ++st) {
+        const long long n = bfills / Cfg::BSTAGES + (st < bfills % Cfg::BSTAGES ? 1 : 0);
+        if (n > 0) wait_drain(b_full + st, static_cast<uint32_t>((n - 1) & 1));
       }
     }
   } else if (warp >= 2 + NE) {
@@ -399,15 +414,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         for (int kb = s.kb0; kb < s.kb1 && ok; kb += Cfg::RK) {
           const int n = s.kb1 - kb < Cfg::RK ? s.kb1 - kb : Cfg::RK;
           if (!wait_bounded(raw_full + rs, rph, abort_flag)) { ok = false; break; }
-          // the A slots of these K blocks are free once the MMAs that read them are done
-          {
-            uint32_t c2 = cs, p2 = cph;
-            for (int c = 0; c < n && ok; ++c) {
-              if (!wait_bounded(empty + c2, p2 ^ 1u, abort_flag)) ok = false;
-              if (++c2 == STAGES) { c2 = 0; p2 ^= 1u; }
-            }
-            if (!ok) break;
-          }
+          // the A stage is free once the MMAs that read it are done
+          if (!wait_bounded(empty + cs, cph ^ 1u, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint8_t* raw = smRaw + rs * Cfg::RAW_BYTES;
           // raw row (128-byte swizzle): K block c is chunks 4(c&1)..4(c&1)+3 of
@@ -430,7 +438,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
             i8x4_to_bf16x4(w1.y, o[10], o[11]);
             i8x4_to_bf16x4(w1.z, o[12], o[13]);
             i8x4_to_bf16x4(w1.w, o[14], o[15]);
-            tmem_st16(a_lane + slot * Cfg::A_TMEM_COLS + half * 16, o);
+            tmem_st16(a_lane + (cs * Cfg::RK + slot) * Cfg::A_TMEM_COLS + half * 16, o);
           };
           if (n == Cfg::RK) {
             uint4 w[Cfg::RK][2];
@@ -440,28 +448,18 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
               w[c][1] = chunk(c, 1);
             }
 #pragma unroll
-            for (int c = 0; c < Cfg::RK; ++c)
-              convert(w[c][0], w[c][1], cs + c >= STAGES ? cs + c - STAGES : cs + c);
+            for (int c = 0; c < Cfg::RK; ++c) convert(w[c][0], w[c][1], c);
           } else {
-            uint32_t c2 = cs;
-            for (int c = 0; c < n; ++c) {
-              convert(chunk(c, 0), chunk(c, 1), c2);
-              if (++c2 == STAGES) c2 = 0;
-            }
+            for (int c = 0; c < n; ++c) convert(chunk(c, 0), chunk(c, 1), c);
           }
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
           if (lane == 0) {
             mbar_arrive(raw_empty + rs);
-            for (int c = 0; c < n; ++c) {
-              mbar_arrive(full + cs);
-              if (++cs == STAGES) { cs = 0; cph ^= 1u; }
-            }
-          } else {
-            for (int c = 0; c < n; ++c)
-              if (++cs == STAGES) { cs = 0; cph ^= 1u; }
+            mbar_arrive(full + cs);
           }
+          if (++cs == STAGES) { cs = 0; cph ^= 1u; }
           if (++rs == Cfg::RSTAGES) { rs = 0; rph ^= 1u; }
         }
       }
@@ -536,6 +534,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     if (lane == 0) {
       const uint32_t idesc = Cfg::I8 ? idesc_i8_s32(BN) : idesc_bf16_f32(BN);
       uint32_t stage = 0, phase = 0;
+      uint32_t bstage = 0, bphase = 0;  // CONV: the separate B ring
       uint32_t local = 0;
       SegIter it;
       it.init(g);
@@ -559,6 +558,36 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
             mma_commit(tfull + p);
             if (++stage == STAGES) { stage = 0; phase ^= 1u; }
           }
+        } else if constexpr (Cfg::CONV) {
+          // groups of RK K blocks: A from tensor memory, B from its ring,
+          // one commit per group
+          const uint32_t a = local % NACC, u = local / NACC;
+          if (!wait_bounded(tempty + a, (u & 1u) ^ 1u, abort_flag)) break;
+          tc_fence_after();
+          int i = 0;  // K block index within the segment
+          for (int kb = s.kb0; kb < s.kb1; kb += Cfg::RK) {
+            const int n = s.kb1 - kb < Cfg::RK ? s.kb1 - kb : Cfg::RK;
+            if (!wait_bounded(full + stage, phase, abort_flag)) { ok = false; break; }
+            if (!wait_bounded(b_full + bstage, bphase, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t a_col = tmem + Cfg::ACC_COLS + stage * Cfg::RK * Cfg::A_TMEM_COLS;
+            const uint32_t sb0 = smem_u32(smB + bstage * Cfg::RK * Cfg::B_BYTES);
+            for (int c = 0; c < n; ++c, ++i) {
+              const uint32_t d = tmem + (a * Cfg::NSUB + i % Cfg::NSUB) * BN;
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                mma_bf16_tmem_a(d, a_col + c * Cfg::A_TMEM_COLS + k * 8,
+                                smem_desc_sw128(sb0 + c * Cfg::B_BYTES + k * 32), idesc,
+                                (i >= Cfg::NSUB || k > 0) ? 1u : 0u);
+            }
+            mma_commit(empty + stage);
+            mma_commit(b_empty + bstage);
+            if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+            if (++bstage == Cfg::BSTAGES) { bstage = 0; bphase ^= 1u; }
+          }
+          if (!ok) break;
+          mma_commit(tfull + a);
+          ++local;
         } else {
           const uint32_t a = local % NACC, u = local / NACC;
           if (!wait_bounded(tempty + a, (u & 1u) ^ 1u, abort_flag)) break;
@@ -573,10 +602,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
               const uint32_t accum = (i >= Cfg::NSUB || k > 0) ? 1u : 0u;
-              if constexpr (Cfg::CONV)
-                mma_bf16_tmem_a(d, tmem + Cfg::ACC_COLS + stage * Cfg::A_TMEM_COLS + k * 8,
-                                smem_desc_sw128(sb + k * 32), idesc, accum);
-              else if constexpr (Cfg::I8)
+              if constexpr (Cfg::I8)
                 mma_i8(d, smem_desc_sw128(sa + k * 32), smem_desc_sw128(sb + k * 32), idesc, accum);
               else
                 mma_bf16(d, smem_desc_sw128(sa + k * 32), smem_desc_sw128(sb + k * 32), idesc,

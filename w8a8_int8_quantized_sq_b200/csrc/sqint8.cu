@@ -312,9 +312,9 @@ sq_status run_gemm(GemmKind kind, const void* act, const void* wt, const float* 
       return launch_gemm<GemmCfg<false, 256, 4, false, EPI_SCALE>>(ta, tb, g, p.grid, st, pdl);
     case GK_W8A16_CONV:
       if (p.bn == 16)
-        return launch_gemm<GemmCfg<false, 16, 12, true, EPI_SCALE, true, 5>>(ta, tb, g, p.grid,
-                                                                            st, pdl);
-      return launch_gemm<GemmCfg<false, 32, 8, true, EPI_SCALE, true, 5>>(ta, tb, g, p.grid, st,
+        return launch_gemm<GemmCfg<false, 16, 3, true, EPI_SCALE, true, 5>>(ta, tb, g, p.grid,
+                                                                           st, pdl);
+      return launch_gemm<GemmCfg<false, 32, 2, true, EPI_SCALE, true, 5>>(ta, tb, g, p.grid, st,
                                                                          pdl);
   }
   return SQ_ERR_SHAPE;
