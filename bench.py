@@ -426,25 +426,32 @@ def profile_case(args):
     x = inputs.gen_x(M, K, inputs.SEED_BASE + 100,
                      inputs.XRecipe(col_count=max(1, K // 100), col_factor=30.0)).to(dev)
     w = inputs.gen_w(N, K, inputs.SEED_BASE + 100).to(dev)
+    # enough weight copies, used in turn, that no call finds its weights in L2
+    l2 = 126 * 2 ** 20
+    copies = max(2, -(-3 * l2 // (N * K)))
     if args.profile == "w8a8":
         s, inv = sq.smooth_factors(x, w)
         q_w, s_ch = sq.quant_weight(w, s)
-        fn = lambda: sq.linear_w8a8(x, inv, q_w, s_ch)  # noqa: E731
+        q_ws = [q_w] + [q_w.clone() for _ in range(copies - 1)]
+        fn = lambda i: sq.linear_w8a8(x, inv, q_ws[i % copies], s_ch)  # noqa: E731
     elif args.profile == "gs128":
         q_w, s_blk = sq.quant_weight(w, None, group=128)
         q_a, s_tok = sq.quant_per_token(x, None)
-        fn = lambda: sq.w8a8_gs128_mm(q_a, s_tok, q_w, s_blk)  # noqa: E731
+        q_ws = [q_w] + [q_w.clone() for _ in range(copies - 1)]
+        fn = lambda i: sq.w8a8_gs128_mm(q_a, s_tok, q_ws[i % copies], s_blk)  # noqa: E731
     else:
         q_w, s_ch = sq.quant_weight(w, None)
-        fn = lambda: sq.w8a16_mm(x, q_w, s_ch)  # noqa: E731
+        q_ws = [q_w] + [q_w.clone() for _ in range(copies - 1)]
+        fn = lambda i: sq.w8a16_mm(x, q_ws[i % copies], s_ch)  # noqa: E731
     del w
-    for _ in range(args.warmup):
-        fn()
+    for i in range(args.warmup):
+        fn(i)
     torch.cuda.synchronize()
-    t_eager = time_batches(lambda i: fn(), args.steps, warmup=0)
-    t_graph = time_graph(lambda i: fn(), args.steps, reps=3)
+    t_eager = time_batches(fn, args.steps, warmup=0)
+    t_graph = time_graph(fn, args.steps, reps=3)
     print(json.dumps({"profile": args.profile, "M": M, "N": N, "K": K, "steps": args.steps,
-                      "ms_per_call": t_graph * 1e3, "ms_per_call_eager": t_eager * 1e3}),
+                      "weight_copies": copies, "ms_per_call": t_graph * 1e3,
+                      "ms_per_call_eager": t_eager * 1e3}),
           flush=True)
     return 0
 

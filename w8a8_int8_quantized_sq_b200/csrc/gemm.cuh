@@ -63,8 +63,8 @@ __host__ __device__ constexpr int pow2_at_least(int v) {
 // and write it straight into a ring of STAGES A tiles in tensor memory
 // (tcgen05.st; 32 columns of two bf16 per 128-lane row per K block), then wait
 // for their stores once and release the raw stage; the MMA reads A from tensor
-// memory.  A second producer thread loads the K blocks' B tiles into their own
-// shared-memory ring.  Everything moves in groups of RK K blocks (one raw
+// memory.  A producer warp of its own loads the K blocks' B tiles into their
+// own shared-memory ring.  Everything moves in groups of RK K blocks (one raw
 // stage, one A stage, one B stage): one hand-off and one tcgen05.commit per
 // 4 x RK MMAs, because short N = 16 MMAs committed one K block at a time keep
 // the tensor pipe waiting on each commit.  Keeping A out of shared
@@ -92,7 +92,8 @@ struct GemmCfg {
   static constexpr int RAW_BYTES = RAW_A_BYTES;
   static constexpr int NE = (EPI == EPI_GS128) ? 8 : 4;  // epilogue warps
   static constexpr int NCV = CONV ? 8 : 0;               // converter warps (2 per row)
-  static constexpr int THREADS = 64 + NE * 32 + NCV * 32;
+  // CONV: one more warp, the producer of the B tiles (warp 2 + NE + NCV)
+  static constexpr int THREADS = 64 + NE * 32 + NCV * 32 + (CONV ? 32 : 0);
   static constexpr int NACC = (EPI == EPI_GS128) ? 4 : 2;
   // Narrow (swapped, small-token) tiles rotate the K blocks over NSUB
   // independent accumulators, so consecutive tiny MMAs do not wait on each
@@ -178,7 +179,8 @@ struct SegIter {
 // policy != 0: the 16-byte BF16 output stores carry that L2 eviction hint.
 template <class Cfg>
 __device__ __forceinline__ void store_chunk(const GemmArgs& g, int rt, int ct, int rr, int c0,
-                                            const uint32_t (&v)[Cfg::CW], uint64_t policy = 0) {
+                                            const uint32_t (&v)[Cfg::CW], uint64_t policy = 0,
+                                            const float* sc_pre = nullptr) {
   constexpr int CW = Cfg::CW;
   const int r = rt * Cfg::BM + rr;
   const int cb = ct * Cfg::BN + c0;
@@ -230,7 +232,7 @@ __device__ __forceinline__ void store_chunk(const GemmArgs& g, int rt, int ct, i
       }
     } else {
       __nv_bfloat16* out = static_cast<__nv_bfloat16*>(g.out);
-      const float sc = __ldg(g.s_ch + n);
+      const float sc = sc_pre ? *sc_pre : __ldg(g.s_ch + n);
 #pragma unroll
       for (int j = 0; j < CW; ++j) {
         const int m = cb + j;
@@ -340,62 +342,66 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
-  if (warp == 0 && Cfg::CONV) {
-    // ------------------------------- TMA producers: raw int8 weights (lane 0)
-    //                                   and the K blocks' B tiles (lane 1)
-    if (lane == 0) {
-      tma_prefetch_desc(&tmA);
-      uint32_t rs = 0, rph = 0;
-      long long fills = 0;
-      SegIter it;
-      it.init(g);
-      Seg s;
-      bool ok = true;
-      while (ok && it.next(g, s)) {
-        const int rt = s.tile % g.tiles_r;
-        for (int kb = s.kb0; kb < s.kb1; kb += Cfg::RK) {
-          const int n = s.kb1 - kb < Cfg::RK ? s.kb1 - kb : Cfg::RK;  // K blocks used
-          if (!wait_bounded(raw_empty + rs, rph ^ 1u, abort_flag)) { ok = false; break; }
-          uint8_t* st = smRaw + rs * Cfg::RAW_BYTES;
-          const int boxes = (n + 1) / 2;
-          mbar_arrive_expect_tx(raw_full + rs, boxes * Cfg::RAW_BOX_BYTES);
-          // 128 contiguous weight bytes per row per box, both boxes back to back
-          for (int b2 = 0; b2 < boxes; ++b2)
-            tma_load_2d(st + b2 * Cfg::RAW_BOX_BYTES, &tmA, (kb + 2 * b2) * Cfg::KB_ELEMS,
-                        rt * Cfg::BM, raw_full + rs);
-          ++fills;
-          if (++rs == Cfg::RSTAGES) { rs = 0; rph ^= 1u; }
+  if ((warp == 0 || warp == 2 + NE + Cfg::NCV) && Cfg::CONV) {
+    // ------------------------------- TMA producers: raw int8 weights (warp 0)
+    //                          and the K blocks' B tiles (the last warp); one
+    //                          warp each, since two spinning lanes of one warp
+    //                          take turns and starve each other
+    if constexpr (Cfg::CONV) {
+      if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA);
+        uint32_t rs = 0, rph = 0;
+        long long fills = 0;
+        SegIter it;
+        it.init(g);
+        Seg s;
+        bool ok = true;
+        while (ok && it.next(g, s)) {
+          const int rt = s.tile % g.tiles_r;
+          for (int kb = s.kb0; kb < s.kb1; kb += Cfg::RK) {
+            const int n = s.kb1 - kb < Cfg::RK ? s.kb1 - kb : Cfg::RK;  // K blocks used
+            if (!wait_bounded(raw_empty + rs, rph ^ 1u, abort_flag)) { ok = false; break; }
+            uint8_t* st = smRaw + rs * Cfg::RAW_BYTES;
+            const int boxes = (n + 1) / 2;
+            mbar_arrive_expect_tx(raw_full + rs, boxes * Cfg::RAW_BOX_BYTES);
+            // 128 contiguous weight bytes per row per box, both boxes back to back
+            for (int b2 = 0; b2 < boxes; ++b2)
+              tma_load_2d(st + b2 * Cfg::RAW_BOX_BYTES, &tmA, (kb + 2 * b2) * Cfg::KB_ELEMS,
+                          rt * Cfg::BM, raw_full + rs);
+            ++fills;
+            if (++rs == Cfg::RSTAGES) { rs = 0; rph ^= 1u; }
+          }
         }
-      }
-      for (int st = 0; st < Cfg::RSTAGES; ++st) {
-        const long long n = fills / Cfg::RSTAGES + (st < fills % Cfg::RSTAGES ? 1 : 0);
-        if (n > 0) wait_drain(raw_full + st, static_cast<uint32_t>((n - 1) & 1));
-      }
-    } else if (lane == 1) {
-      tma_prefetch_desc(&tmB);
-      griddep_wait();  // the activations may come from the preceding kernel
-      uint32_t cs = 0, cph = 0;
-      long long bfills = 0;
-      SegIter it;
-      it.init(g);
-      Seg s;
-      bool ok = true;
-      while (ok && it.next(g, s)) {
-        const int ct = s.tile / g.tiles_r;
-        for (int kb = s.kb0; kb < s.kb1; kb += Cfg::RK) {
-          const int n = s.kb1 - kb < Cfg::RK ? s.kb1 - kb : Cfg::RK;
-          if (!wait_bounded(b_empty + cs, cph ^ 1u, abort_flag)) { ok = false; break; }
-          mbar_arrive_expect_tx(b_full + cs, n * Cfg::B_BYTES);
-          for (int c = 0; c < n; ++c)
-            tma_load_2d(smB + (cs * Cfg::RK + c) * Cfg::B_BYTES, &tmB, (kb + c) * Cfg::KB_ELEMS,
-                        ct * BN, b_full + cs);
-          ++bfills;
-          if (++cs == Cfg::BSTAGES) { cs = 0; cph ^= 1u; }
+        for (int st = 0; st < Cfg::RSTAGES; ++st) {
+          const long long n = fills / Cfg::RSTAGES + (st < fills % Cfg::RSTAGES ? 1 : 0);
+          if (n > 0) wait_drain(raw_full + st, static_cast<uint32_t>((n - 1) & 1));
         }
-      }
-      for (int st = 0; st < Cfg::BSTAGES; ++st) {
-        const long long n = bfills / Cfg::BSTAGES + (st < bfills % Cfg::BSTAGES ? 1 : 0);
-        if (n > 0) wait_drain(b_full + st, static_cast<uint32_t>((n - 1) & 1));
+      } else if (warp != 0 && lane == 0) {
+        tma_prefetch_desc(&tmB);
+        griddep_wait();  // the activations may come from the preceding kernel
+        uint32_t cs = 0, cph = 0;
+        long long bfills = 0;
+        SegIter it;
+        it.init(g);
+        Seg s;
+        bool ok = true;
+        while (ok && it.next(g, s)) {
+          const int ct = s.tile / g.tiles_r;
+          for (int kb = s.kb0; kb < s.kb1; kb += Cfg::RK) {
+            const int n = s.kb1 - kb < Cfg::RK ? s.kb1 - kb : Cfg::RK;
+            if (!wait_bounded(b_empty + cs, cph ^ 1u, abort_flag)) { ok = false; break; }
+            mbar_arrive_expect_tx(b_full + cs, n * Cfg::B_BYTES);
+            for (int c = 0; c < n; ++c)
+              tma_load_2d(smB + (cs * Cfg::RK + c) * Cfg::B_BYTES, &tmB, (kb + c) * Cfg::KB_ELEMS,
+                          ct * BN, b_full + cs);
+            ++bfills;
+            if (++cs == Cfg::BSTAGES) { cs = 0; cph ^= 1u; }
+          }
+        }
+        for (int st = 0; st < Cfg::BSTAGES; ++st) {
+          const long long n = bfills / Cfg::BSTAGES + (st < bfills % Cfg::BSTAGES ? 1 : 0);
+          if (n > 0) wait_drain(b_full + st, static_cast<uint32_t>((n - 1) & 1));
+        }
       }
     }
   } else if (warp >= 2 + NE) {
@@ -531,7 +537,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    // The whole warp runs the loop and waits; one elected lane issues the
+    // MMAs and commits.
+    {
       const uint32_t idesc = Cfg::I8 ? idesc_i8_s32(BN) : idesc_bf16_f32(BN);
       uint32_t stage = 0, phase = 0;
       uint32_t bstage = 0, bphase = 0;  // CONV: the separate B ring
@@ -544,81 +552,96 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         if constexpr (Cfg::EPI == EPI_GS128) {
           for (int kb = s.kb0; kb < s.kb1 && ok; ++kb, ++local) {
             const uint32_t p = local % NACC, u = local / NACC;
-            if (!wait_bounded(tempty + p, u & 1u, abort_flag)) { ok = false; break; }
+            if (!warp_wait_bounded(tempty + p, u & 1u, abort_flag)) { ok = false; break; }
             tc_fence_after();
-            if (!wait_bounded(full + stage, phase, abort_flag)) { ok = false; break; }
+            if (!warp_wait_bounded(full + stage, phase, abort_flag)) { ok = false; break; }
             tc_fence_after();
             const uint32_t sa = smem_u32(smA + stage * Cfg::A_BYTES);
             const uint32_t sb = smem_u32(smB + stage * Cfg::B_BYTES);
+            if (elect_one()) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-              mma_i8(tmem + p * BN, smem_desc_sw128(sa + k * 32), smem_desc_sw128(sb + k * 32),
-                     idesc, 1u);
-            mma_commit(empty + stage);
-            mma_commit(tfull + p);
+              for (int k = 0; k < 4; ++k)
+                mma_i8(tmem + p * BN, smem_desc_sw128(sa + k * 32), smem_desc_sw128(sb + k * 32),
+                       idesc, 1u);
+              mma_commit(empty + stage);
+              mma_commit(tfull + p);
+            }
+            __syncwarp();
             if (++stage == STAGES) { stage = 0; phase ^= 1u; }
           }
         } else if constexpr (Cfg::CONV) {
           // groups of RK K blocks: A from tensor memory, B from its ring,
           // one commit per group
           const uint32_t a = local % NACC, u = local / NACC;
-          if (!wait_bounded(tempty + a, (u & 1u) ^ 1u, abort_flag)) break;
+          if (!warp_wait_bounded(tempty + a, (u & 1u) ^ 1u, abort_flag)) break;
           tc_fence_after();
           int i = 0;  // K block index within the segment
           for (int kb = s.kb0; kb < s.kb1; kb += Cfg::RK) {
             const int n = s.kb1 - kb < Cfg::RK ? s.kb1 - kb : Cfg::RK;
-            if (!wait_bounded(full + stage, phase, abort_flag)) { ok = false; break; }
-            if (!wait_bounded(b_full + bstage, bphase, abort_flag)) { ok = false; break; }
+            if (!warp_wait_bounded(full + stage, phase, abort_flag)) { ok = false; break; }
+            if (!warp_wait_bounded(b_full + bstage, bphase, abort_flag)) { ok = false; break; }
             tc_fence_after();
             const uint32_t a_col = tmem + Cfg::ACC_COLS + stage * Cfg::RK * Cfg::A_TMEM_COLS;
             const uint32_t sb0 = smem_u32(smB + bstage * Cfg::RK * Cfg::B_BYTES);
-            for (int c = 0; c < n; ++c, ++i) {
-              const uint32_t d = tmem + (a * Cfg::NSUB + i % Cfg::NSUB) * BN;
+            if (elect_one()) {
+              for (int c = 0; c < n; ++c) {
+                const uint32_t d = tmem + (a * Cfg::NSUB + (i + c) % Cfg::NSUB) * BN;
 #pragma unroll
-              for (int k = 0; k < 4; ++k)
-                mma_bf16_tmem_a(d, a_col + c * Cfg::A_TMEM_COLS + k * 8,
-                                smem_desc_sw128(sb0 + c * Cfg::B_BYTES + k * 32), idesc,
-                                (i >= Cfg::NSUB || k > 0) ? 1u : 0u);
+                for (int k = 0; k < 4; ++k)
+                  mma_bf16_tmem_a(d, a_col + c * Cfg::A_TMEM_COLS + k * 8,
+                                  smem_desc_sw128(sb0 + c * Cfg::B_BYTES + k * 32), idesc,
+                                  (i + c >= Cfg::NSUB || k > 0) ? 1u : 0u);
+              }
+              mma_commit(empty + stage);
+              mma_commit(b_empty + bstage);
             }
-            mma_commit(empty + stage);
-            mma_commit(b_empty + bstage);
+            __syncwarp();
+            i += n;
             if (++stage == STAGES) { stage = 0; phase ^= 1u; }
             if (++bstage == Cfg::BSTAGES) { bstage = 0; bphase ^= 1u; }
           }
           if (!ok) break;
-          mma_commit(tfull + a);
+          if (elect_one()) mma_commit(tfull + a);
+          __syncwarp();
           ++local;
         } else {
           const uint32_t a = local % NACC, u = local / NACC;
-          if (!wait_bounded(tempty + a, (u & 1u) ^ 1u, abort_flag)) break;
+          if (!warp_wait_bounded(tempty + a, (u & 1u) ^ 1u, abort_flag)) break;
           tc_fence_after();
           for (int kb = s.kb0; kb < s.kb1; ++kb) {
-            if (!wait_bounded(full + stage, phase, abort_flag)) { ok = false; break; }
+            if (!warp_wait_bounded(full + stage, phase, abort_flag)) { ok = false; break; }
             tc_fence_after();
             const uint32_t sa = smem_u32(smA + stage * Cfg::A_BYTES);
             const uint32_t sb = smem_u32(smB + stage * Cfg::B_BYTES);
             const int i = kb - s.kb0;
             const uint32_t d = tmem + (a * Cfg::NSUB + i % Cfg::NSUB) * BN;
+            if (elect_one()) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const uint32_t accum = (i >= Cfg::NSUB || k > 0) ? 1u : 0u;
-              if constexpr (Cfg::I8)
-                mma_i8(d, smem_desc_sw128(sa + k * 32), smem_desc_sw128(sb + k * 32), idesc, accum);
-              else
-                mma_bf16(d, smem_desc_sw128(sa + k * 32), smem_desc_sw128(sb + k * 32), idesc,
+              for (int k = 0; k < 4; ++k) {
+                const uint32_t accum = (i >= Cfg::NSUB || k > 0) ? 1u : 0u;
+                if constexpr (Cfg::I8)
+                  mma_i8(d, smem_desc_sw128(sa + k * 32), smem_desc_sw128(sb + k * 32), idesc,
                          accum);
+                else
+                  mma_bf16(d, smem_desc_sw128(sa + k * 32), smem_desc_sw128(sb + k * 32), idesc,
+                           accum);
+              }
+              mma_commit(empty + stage);
             }
-            mma_commit(empty + stage);
+            __syncwarp();
             if (++stage == STAGES) { stage = 0; phase ^= 1u; }
           }
           if (!ok) break;
-          mma_commit(tfull + a);
+          if (elect_one()) mma_commit(tfull + a);
+          __syncwarp();
           ++local;
         }
       }
-      // every MMA issued by this thread has finished before TMEM is freed
-      mma_commit(drain);
-      wait_drain(drain, 0);
+      // every MMA issued by the elected lane has finished before TMEM is freed
+      if (elect_one()) {
+        mma_commit(drain);
+        wait_drain(drain, 0);
+      }
     }
     __syncwarp();
   } else {
@@ -707,12 +730,21 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     } else {
       uint32_t local = 0;
       const long long G = gridDim.x, T = g.total_iters;
+      const int me = blockIdx.x;
       while (it.next(g, s)) {
         const uint32_t a = local % NACC, u = local / NACC;
+        const int rt = s.tile % g.tiles_r, ct = s.tile / g.tiles_r;
+        // the channel scale of this thread's output row, fetched while the
+        // MMAs finish (swapped layout: one weight row per thread)
+        float sc_pre = 0.0f;
+        if constexpr (Cfg::SWAP && Cfg::EPI == EPI_SCALE) {
+          const int n = rt * Cfg::BM + rr;
+          if (n < g.N) sc_pre = __ldg(g.s_ch + n);
+        }
+        const float* scp = (Cfg::SWAP && Cfg::EPI == EPI_SCALE) ? &sc_pre : nullptr;
         const bool w_ok = wait_bounded(tfull + a, u & 1u, abort_flag);
         if (named_bar_or(1, nthr, !w_ok)) break;
         tc_fence_after();
-        const int rt = s.tile % g.tiles_r, ct = s.tile / g.tiles_r;
         const uint32_t tb = lane_base + a * Cfg::NSUB * BN;
         const int nsub = s.kb1 - s.kb0 < Cfg::NSUB ? s.kb1 - s.kb0 : Cfg::NSUB;
         if (s.kb0 == 0 && s.kb1 == g.kb_total) {
@@ -720,15 +752,18 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           for (int c = 0; c < BN; c += CW) {
             uint32_t v[CW];
             tmem_ld_acc<Cfg>(tb, c, nsub, v);
-            store_chunk<Cfg>(g, rt, ct, rr, c, v);
+            store_chunk<Cfg>(g, rt, ct, rr, c, v, 0, scp);
           }
         } else {
           // stream-K part of a tile: publish, count, and the last arrival reduces
           const long long it0 = static_cast<long long>(s.tile) * g.kb_total;
-          const long long b_lo = sk_owner(it0, G, T);
-          const long long b_hi = sk_owner(it0 + g.kb_total - 1, G, T);
-          const int slot = sk_start(blockIdx.x, G, T) >= it0 ? 0 : 1;
-          uint32_t* wrow = g.ws + (static_cast<size_t>(blockIdx.x * 2 + slot) * Cfg::BM + rr) * BN;
+          const int b_lo = static_cast<int>(sk_owner(it0, G, T));
+          const int b_hi = static_cast<int>(sk_owner(it0 + g.kb_total - 1, G, T));
+          // slot 0: a CTA's first segment, 1: its last one.  Only the first
+          // part of a tile can have started in an earlier tile.
+          const int lo_slot = sk_start(b_lo, G, T) < it0 ? 1 : 0;
+          const int slot = me == b_lo ? lo_slot : 0;
+          uint32_t* wrow = g.ws + (static_cast<size_t>(me * 2 + slot) * Cfg::BM + rr) * BN;
 #pragma unroll 1
           for (int c = 0; c < BN; c += CW) {
             uint32_t v[CW];
@@ -755,13 +790,13 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
               for (int j = 0; j < CW; ++j) v[j] = 0u;
               // parts are summed in CTA order; up to NB parts' loads in flight
               constexpr int NB = CW >= 32 ? 2 : 4;
-              for (long long b0 = b_lo; b0 <= b_hi; b0 += NB) {
+              for (int b0 = b_lo; b0 <= b_hi; b0 += NB) {
                 int4 w[NB][CW / 4];
 #pragma unroll
                 for (int u = 0; u < NB; ++u) {
-                  const long long b = b0 + u;
+                  const int b = b0 + u;
                   if (b <= b_hi) {
-                    const int sl = sk_start(b, G, T) >= it0 ? 0 : 1;
+                    const int sl = b == b_lo ? lo_slot : 0;
                     const uint32_t* prow =
                         g.ws + (static_cast<size_t>(b * 2 + sl) * Cfg::BM + rr) * BN + c;
 #pragma unroll
@@ -790,7 +825,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                   }
                 }
               }
-              store_chunk<Cfg>(g, rt, ct, rr, c, v);
+              store_chunk<Cfg>(g, rt, ct, rr, c, v, 0, scp);
             }
           }
         }

@@ -162,37 +162,44 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     }
   } else if (warp == 1) {
     // ----------------------------------------------- MMA issuer (leader)
-    if (leader && lane == 0) {
+    // The whole warp runs the loop; one elected lane issues and commits.
+    if (leader) {
       const uint32_t idesc = Cfg::I8 ? idesc_i8_s32_m256(BN) : idesc_bf16_f32_m256(BN);
       uint32_t stage = 0, phase = 0, local = 0;
       bool ok = true;
       for (int t = cluster; ok && t < g.num_tiles; t += nclusters, ++local) {
         const uint32_t a = local % NACC, u = local / NACC;
-        if (!wait_bounded(tempty + a, (u & 1u) ^ 1u, abort_flag)) break;
+        if (!warp_wait_bounded(tempty + a, (u & 1u) ^ 1u, abort_flag)) break;
         tc_fence_after();
         const uint32_t d = tmem + a * BN;
         for (int kb = 0; kb < g.kb_total; ++kb) {
-          if (!wait_bounded(full + stage, phase, abort_flag)) { ok = false; break; }
+          if (!warp_wait_bounded(full + stage, phase, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = smem_u32(smA + stage * Cfg::A_BYTES);
           const uint32_t sb = smem_u32(smB + stage * Cfg::B_BYTES);
+          if (elect_one()) {
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            if constexpr (Cfg::I8)
-              mma_i8_pair(d, smem_desc_sw128(sa + k * 32), smem_desc_sw128(sb + k * 32), idesc,
-                          (kb > 0 || k > 0) ? 1u : 0u);
-            else
-              mma_bf16_pair(d, smem_desc_sw128(sa + k * 32), smem_desc_sw128(sb + k * 32), idesc,
+            for (int k = 0; k < 4; ++k) {
+              if constexpr (Cfg::I8)
+                mma_i8_pair(d, smem_desc_sw128(sa + k * 32), smem_desc_sw128(sb + k * 32), idesc,
                             (kb > 0 || k > 0) ? 1u : 0u);
+              else
+                mma_bf16_pair(d, smem_desc_sw128(sa + k * 32), smem_desc_sw128(sb + k * 32),
+                              idesc, (kb > 0 || k > 0) ? 1u : 0u);
+            }
+            mma_commit_pair_both(empty + stage);
           }
-          mma_commit_pair_both(empty + stage);
+          __syncwarp();
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
-        mma_commit_pair_both(tfull + a);
+        if (elect_one()) mma_commit_pair_both(tfull + a);
+        __syncwarp();
       }
-      mma_commit_pair(drain);
-      wait_drain(drain, 0);
+      if (elect_one()) {
+        mma_commit_pair(drain);
+        wait_drain(drain, 0);
+      }
     }
     __syncwarp();
   } else {

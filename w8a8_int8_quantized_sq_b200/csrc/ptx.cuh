@@ -90,6 +90,25 @@ __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity,
   }
 }
 
+// wait_bounded for a whole warp: every lane waits, and every lane gets the
+// same answer (false if any lane gave up), so the warp stays converged.
+__device__ __forceinline__ bool warp_wait_bounded(uint64_t* bar, uint32_t parity,
+                                                  volatile int* abort_flag) {
+  return __all_sync(0xffffffffu, wait_bounded(bar, parity, abort_flag));
+}
+
+// One lane of a converged warp; the same lane every time for a full warp.
+// Issuing tcgen05.mma from a converged warp through elect.sync lets the
+// operands stay in uniform registers: a lone lane-0 loop issues about half
+// as fast.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 // Same, ignoring the abort flag: used to drain copies and MMAs already in
 // flight before the CTA exits.
 __device__ __forceinline__ bool wait_drain(uint64_t* bar, uint32_t parity) {
