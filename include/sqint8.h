@@ -154,6 +154,21 @@ sq_status sq_smooth_factors(const void* x_bf16, int64_t M, const void* w_bf16, i
 sq_status sq_quant_weight(const void* w_bf16, const float* smooth, int8_t* q_w, float* scales,
                           int64_t N, int64_t K, int64_t group, void* stream);
 
+/* Launch policy ---------------------------------------------------------- */
+
+/* Overlap of consecutive kernels (programmatic dependent launch; the pages
+ * have no counterpart: it is a launch policy of this library).  enable != 0:
+ * from now on, in this process, w8a8_scaled_mm, w8a8_mm_i32, w8a8_gs128_mm
+ * and w8a16_mm (M <= 32) launch their GEMM so that it may start while the
+ * kernel before it on the stream is still running: it requests its WEIGHT
+ * tiles (q_w) at once and reads everything else (activations, scales,
+ * workspace, output) only after that kernel has completed.  Enable it only
+ * if no kernel that directly precedes such a call on its stream writes that
+ * call's q_w.  enable == 0 (the default): every launch waits for the
+ * preceding work as usual.  sq_w8a8_linear always overlaps its GEMM with its
+ * own quantisation kernel.  Always returns SQ_OK. */
+sq_status sq_set_overlap(int enable);
+
 /* Diagnostics ------------------------------------------------------------ */
 
 /* Synchronises the current device, then returns SQ_ERR_TIMEOUT if any kernel

@@ -265,3 +265,54 @@ def test_fused_linear_pdl(M, N, K):
     for _ in range(3):  # back-to-back calls overlap one call's GEMM with the next quant
         y = sq.linear_w8a8(xd, invd, qwd, schd)
     assert_same(y, ref, "fused linear")
+
+
+# ------------------------------------------------ overlapped (PDL) launches
+
+@pytest.mark.parametrize("op", ["w8a8", "i32", "gs128", "w8a16"])
+def test_overlap_launch_policy(op):
+    """sq_set_overlap(1): each GEMM is launched as a programmatic dependent of
+    the call before it (weights requested before that call ends).  A chain of
+    back-to-back calls on different weights gives exactly the results of
+    ordinary launches, and the first matches the oracle."""
+    M, N, K = (8, 1024, 2048) if op != "w8a16" else (16, 1024, 4096)
+    x = inputs.gen_x(M, K, 23, inputs.XRecipe(col_count=3, col_factor=30.0))
+    ws = [inputs.gen_w(N, K, 40 + i) for i in range(3)]
+    q_a, s_tok = oracle.quant_per_token(x, None)
+    if op == "gs128":
+        qs = [oracle.quant_weight(w, None, group=128) for w in ws]
+    else:
+        qs = [oracle.quant_weight(w, None) for w in ws]
+    xd, qad, std = x.cuda(), q_a.cuda(), s_tok.cuda()
+    qsd = [(q.cuda(), s.cuda()) for q, s in qs]
+
+    def call(i):
+        q_w, sc = qsd[i % 3]
+        if op == "w8a8":
+            return sq.w8a8_scaled_mm(qad, std, q_w, sc)
+        if op == "i32":
+            return sq.w8a8_mm_i32(qad, q_w)
+        if op == "gs128":
+            return sq.w8a8_gs128_mm(qad, std, q_w, sc)
+        return sq.w8a16_mm(xd, q_w, sc)
+
+    plain = [call(i) for i in range(6)]
+    torch.cuda.synchronize()
+    sq.set_overlap(True)
+    try:
+        over = [call(i) for i in range(6)]
+        torch.cuda.synchronize()
+    finally:
+        sq.set_overlap(False)
+    for i in range(6):
+        assert_same(over[i], plain[i].cpu(), f"{op} call {i}")
+    q_w, sc = qs[0]
+    if op == "w8a8":
+        assert_same(plain[0], oracle.w8a8_scaled_mm(q_a, s_tok, q_w, sc), "w8a8 vs oracle")
+    elif op == "i32":
+        assert_same(plain[0], oracle.mm_i32(q_a, q_w), "i32 vs oracle")
+    elif op == "gs128":
+        assert_same(plain[0], oracle.gs128_mm(q_a, s_tok, q_w, sc), "gs128 vs oracle")
+    else:
+        _check_w8a16(x, q_w, sc)
+    sq.check_device_error()

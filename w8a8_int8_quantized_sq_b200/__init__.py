@@ -65,6 +65,7 @@ def lib() -> ctypes.CDLL:
                 "sq_smooth_factors": [vp, i64, vp, i64, i64, dbl, dbl, vp, vp, vp],
                 "sq_quant_weight": [vp, vp, vp, vp, i64, i64, i64, vp],
                 "sq_check_device_error": [ctypes.c_int],
+                "sq_set_overlap": [ctypes.c_int],
             }
             for name, args in sig.items():
                 f = getattr(L, name)
@@ -81,7 +82,7 @@ def lib() -> ctypes.CDLL:
 EXPORTS = ("sq_quant_per_token", "w8a8_scaled_mm", "w8a8_gs128_mm", "w8a16_mm",
            "sq_workspace_bytes", "w8a8_mm_i32", "sq_smooth_factors", "sq_quant_weight",
            "sq_check_device_error", "sq_status_string", "w8a8_scaled_mm_noalloc",
-           "sq_w8a8_linear")
+           "sq_w8a8_linear", "sq_set_overlap")
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -223,6 +224,14 @@ def quant_weight(w, smooth: Optional[torch.Tensor] = None, group: int = 0):
     _check("sq_quant_weight", lib().sq_quant_weight(
         _ptr(w), _ptr(smooth), _ptr(q), _ptr(sc), N, K, group, _stream(w.device)))
     return q, sc
+
+
+def set_overlap(enable: bool) -> None:
+    """Process-wide launch policy (sq_set_overlap): when on, the GEMM entry
+    points may start streaming their weights while the preceding kernel on the
+    stream still runs.  Only for callers whose preceding kernel never writes
+    the weights of the next call."""
+    _check("sq_set_overlap", lib().sq_set_overlap(1 if enable else 0))
 
 
 def check_device_error(reset: bool = True) -> None:

@@ -341,6 +341,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  // a programmatic dependent of this grid may be scheduled now; it waits for
+  // this grid's completion before it reads anything this grid writes
+  griddep_launch_dependents();
 
   if ((warp == 0 || warp == 2 + NE + Cfg::NCV) && Cfg::CONV) {
     // ------------------------------- TMA producers: raw int8 weights (warp 0)

@@ -97,6 +97,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   cluster_sync();  // barriers of both CTAs initialised, tensor memory allocated in both
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  griddep_launch_dependents();  // dependents wait for this grid's completion
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer

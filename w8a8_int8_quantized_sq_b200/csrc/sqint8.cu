@@ -113,6 +113,11 @@ bool pair_enabled() {
   return on;
 }
 
+// sq_set_overlap: GEMM launches become programmatic dependents of the
+// preceding kernel on the stream (they request weights before that kernel ends).
+std::atomic<int> g_overlap{0};
+bool overlap_on() { return g_overlap.load(std::memory_order_relaxed) != 0; }
+
 GemmPlan plan_gemm(GemmKind kind, int64_t M, int64_t N, int64_t K, int sms) {
   GemmPlan p{};
   const bool i8 = kind != GK_BF16 && kind != GK_W8A16_CONV;
@@ -507,7 +512,7 @@ sq_status w8a8_scaled_mm(const int8_t* q_a, const float* s_tok, const int8_t* q_
       !aligned16(y_bf16))
     return SQ_ERR_ALIGN;
   return run_gemm(GK_I8_SCALE, q_a, q_w, s_tok, s_ch, nullptr, y_bf16, M, N, K, workspace,
-                  ws_bytes, static_cast<cudaStream_t>(stream));
+                  ws_bytes, static_cast<cudaStream_t>(stream), overlap_on());
 }
 
 sq_status sq_w8a8_linear(const void* x_bf16, const float* inv_smooth, const int8_t* q_w,
@@ -539,7 +544,7 @@ sq_status w8a8_mm_i32(const int8_t* q_a, const int8_t* q_w, int32_t* acc, int64_
   if (!q_a || !q_w || !acc) return SQ_ERR_NULL;
   if (!aligned16(q_a) || !aligned16(q_w) || !aligned16(acc)) return SQ_ERR_ALIGN;
   return run_gemm(GK_I8_I32, q_a, q_w, nullptr, nullptr, nullptr, acc, M, N, K, workspace,
-                  ws_bytes, static_cast<cudaStream_t>(stream));
+                  ws_bytes, static_cast<cudaStream_t>(stream), overlap_on());
 }
 
 sq_status w8a8_gs128_mm(const int8_t* q_a, const float* s_tok, const int8_t* q_w,
@@ -553,7 +558,7 @@ sq_status w8a8_gs128_mm(const int8_t* q_a, const float* s_tok, const int8_t* q_w
       !aligned16(y_bf16))
     return SQ_ERR_ALIGN;
   return run_gemm(GK_GS128, q_a, q_w, s_tok, nullptr, s_blk, y_bf16, M, N, K, workspace,
-                  ws_bytes, static_cast<cudaStream_t>(stream));
+                  ws_bytes, static_cast<cudaStream_t>(stream), overlap_on());
 }
 
 sq_status w8a16_mm(const void* x_bf16, const int8_t* q_w, const float* s_ch, void* y_bf16,
@@ -574,14 +579,20 @@ sq_status w8a16_mm(const void* x_bf16, const int8_t* q_w, const float* s_ch, voi
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (M <= 32)  // weight-read bound: int8 weights are converted on load, in the GEMM
     return run_gemm(GK_W8A16_CONV, x_bf16, q_w, nullptr, s_ch, nullptr, y_bf16, M, N, K,
-                    workspace, ws_bytes, st);
+                    workspace, ws_bytes, st, overlap_on());
   __nv_bfloat16* wb = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(workspace) + w_off);
   const int64_t n16 = N * K / 16;
   const int64_t blocks = (n16 + 255) / 256 < 4 * sms ? (n16 + 255) / 256 : 4 * sms;
   i8_to_bf16_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(q_w, wb, n16);
   if (launch_status() != SQ_OK) return SQ_ERR_CUDA;
+  // never a programmatic launch here: its weights come from the kernel just before
   return run_gemm(GK_BF16, x_bf16, wb, nullptr, s_ch, nullptr, y_bf16, M, N, K, workspace,
                   w_off, st);
+}
+
+sq_status sq_set_overlap(int enable) {
+  g_overlap.store(enable ? 1 : 0, std::memory_order_relaxed);
+  return SQ_OK;
 }
 
 sq_status sq_check_device_error(int reset) {
