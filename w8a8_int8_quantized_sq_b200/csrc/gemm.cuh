@@ -23,11 +23,12 @@
 // the parts in CTA order and runs the epilogue, then resets the counter.
 //
 // EPI_GS128 (group-size-128 weight scales): every 128-wide K block is MMA'd
-// into its own TMEM buffer that starts at the int32 pattern of 1.5 * 2^23,
-// so the block partial P arrives as the float 1.5 * 2^23 + P exactly and one
-// subtraction recovers f32(P); the epilogue warps then accumulate
-// fmaf(f32(P), s_blk[n, kb], acc) in registers in K-block order and restore
-// the buffer's starting pattern for its next use.
+// into a fresh int32 TMEM buffer (4 in rotation).  The epilogue warps load a
+// buffer's 64 columns per thread at once and release it, then convert each
+// block partial P exactly (|P| <= 128 * 127^2 < 2^21: the integer add of the
+// bits of 1.5 * 2^23 puts P in the mantissa, one subtraction leaves f32(P))
+// and accumulate fmaf(f32(P), s_blk[n, kb], acc) in registers in K-block
+// order.
 #pragma once
 #include "ptx.cuh"
 #include "quant.cuh"  // exact int8 -> bf16 conversion
@@ -563,9 +564,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
             const uint32_t sb = smem_u32(smB + stage * Cfg::B_BYTES);
             if (elect_one()) {
 #pragma unroll
-              for (int k = 0; k < 4; ++k)
+              for (int k = 0; k < 4; ++k)  // a fresh int32 accumulator per K block
                 mma_i8(tmem + p * BN, smem_desc_sw128(sa + k * 32), smem_desc_sw128(sb + k * 32),
-                       idesc, 1u);
+                       idesc, k > 0 ? 1u : 0u);
               mma_commit(empty + stage);
               mma_commit(tfull + p);
             }
@@ -663,26 +664,34 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       const int h = ew / 4;
       const int col0 = h * CPT;
       const int et = ew * 32 + lane;
-      // every buffer starts at the bias pattern; releasing it completes phase 0
-#pragma unroll
-      for (int p = 0; p < NACC; ++p)
-#pragma unroll
-        for (int c = 0; c < CPT; c += 32) tmem_st32_const(lane_base + p * BN + col0 + c, 0x4B400000u);
-      tc_fence_before();
-      __syncwarp();
+      // every buffer starts free: releasing it completes phase 0
       if (lane == 0)
         for (int p = 0; p < NACC; ++p) mbar_arrive(tempty + p);
       uint32_t local = 0;
       bool ok = true;
       while (ok && it.next(g, s)) {
         const int rt = s.tile % g.tiles_r, ct = s.tile / g.tiles_r;
-        // stage this tile's block scales, transposed to [kb][n]
+        // stage this tile's block scales, transposed to [kb][n]; each thread
+        // requests a batch of its elements before storing any
         named_bar_sync(1, nthr);
         const int total = g.kb_total * BN;
-        for (int idx = et; idx < total; idx += nthr) {
-          const int j = idx / g.kb_total, kb = idx - j * g.kb_total;
-          const int n = ct * BN + j;
-          sblk[kb * Cfg::SBLK_STRIDE + j] = n < g.N ? __ldg(g.s_blk + static_cast<size_t>(n) * g.kb_total + kb) : 0.0f;
+        for (int base = 0; base < total; base += 8 * nthr) {
+          float vals[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int idx = base + i * nthr + et;
+            const int j = idx / g.kb_total, kb = idx - j * g.kb_total;
+            const int n = ct * BN + j;
+            vals[i] = (idx < total && n < g.N)
+                          ? __ldg(g.s_blk + static_cast<size_t>(n) * g.kb_total + kb)
+                          : 0.0f;
+          }
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int idx = base + i * nthr + et;
+            const int j = idx / g.kb_total, kb = idx - j * g.kb_total;
+            if (idx < total) sblk[kb * Cfg::SBLK_STRIDE + j] = vals[i];
+          }
         }
         named_bar_sync(1, nthr);
         float acc[CPT];
@@ -693,25 +702,27 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           const bool w_ok = wait_bounded(tfull + p, u & 1u, abort_flag);
           if (named_bar_or(1, nthr, !w_ok)) { ok = false; break; }
           tc_fence_after();
-          const float* sk = sblk + kb * Cfg::SBLK_STRIDE + col0;
-#pragma unroll
-          for (int c = 0; c < CPT; c += 32) {
-            uint32_t v[32];
-            const uint32_t ta = lane_base + p * BN + col0 + c;
-            tmem_ld32(ta, v);
-#pragma unroll
-            for (int j = 0; j < 32; j += 4) {
-              const float4 s4 = *reinterpret_cast<const float4*>(sk + c + j);
-              acc[c + j] = __fmaf_rn(__fsub_rn(__uint_as_float(v[j]), 12582912.0f), s4.x, acc[c + j]);
-              acc[c + j + 1] = __fmaf_rn(__fsub_rn(__uint_as_float(v[j + 1]), 12582912.0f), s4.y, acc[c + j + 1]);
-              acc[c + j + 2] = __fmaf_rn(__fsub_rn(__uint_as_float(v[j + 2]), 12582912.0f), s4.z, acc[c + j + 2]);
-              acc[c + j + 3] = __fmaf_rn(__fsub_rn(__uint_as_float(v[j + 3]), 12582912.0f), s4.w, acc[c + j + 3]);
-            }
-            tmem_st32_const(ta, 0x4B400000u);
-          }
+          // this K block's int32 sums (|sum| <= 128 * 127 * 127 < 2^22), then
+          // the buffer goes straight back to the MMA
+          static_assert(CPT == 64, "one 64-column load per K block");
+          uint32_t v[64];
+          tmem_ld64(lane_base + p * BN + col0, v);
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(tempty + p);
+          // exact int32 -> fp32: add the bits of 1.5 * 2^23 (the sum lands in
+          // the mantissa), subtract 1.5 * 2^23; then one rounding per step
+          const float* sk = sblk + kb * Cfg::SBLK_STRIDE + col0;
+#pragma unroll
+          for (int j = 0; j < 64; j += 4) {
+            const float4 s4 = *reinterpret_cast<const float4*>(sk + j);
+            const float sc[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float f = __fsub_rn(__uint_as_float(v[j + i] + 0x4B400000u), 12582912.0f);
+              acc[j + i] = __fmaf_rn(f, sc[i], acc[j + i]);
+            }
+          }
         }
         if (!ok) break;
         const int m = rt * Cfg::BM + rr;
