@@ -95,7 +95,12 @@ def test_mm_i32_configs(cfg):
     assert_same(acc, ref, "int32 acc")
 
 
+# small M: whole K splits combined inside clusters of 2, 3, 5 and 8 CTAs
+# ((16, 128, 256), (7, 144, 384), (17, 272, 640), (24, 3712, 2560),
+# (8, 9472, 2048), (8, 2304, 4096)), or in the workspace when a tile has more
+# splits than a cluster may hold ((32, 128, 1280)) or K is long (stream-K)
 SHAPES = [(1, 16, 128), (7, 144, 384), (16, 128, 256), (17, 272, 640), (32, 128, 1280),
+          (24, 3712, 2560), (8, 9472, 2048), (8, 2304, 4096),
           (33, 256, 256), (129, 400, 384), (300, 528, 1024), (256, 512, 5120)]
 
 

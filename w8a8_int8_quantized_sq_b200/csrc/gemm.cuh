@@ -50,6 +50,8 @@ struct GemmArgs {
   void* out;              // bf16 [M, N] or int32 [M, N]
   uint32_t* ws;           // stream-K slots [grid][2][128][BN] 32-bit words
   unsigned int* ws_cnt;   // stream-K arrival counters [num_tiles]
+  int csplit;             // > 1: the csplit CTAs of a tile form a cluster and
+                          // combine their K parts in distributed shared memory
 };
 
 __host__ __device__ constexpr int pow2_at_least(int v) {
@@ -118,11 +120,15 @@ struct GemmCfg {
   static constexpr int OFF_B = OFF_A + STAGES * A_SMEM_BYTES;
   static constexpr int OFF_BAR = OFF_B + B_RING_BYTES;
   static constexpr int NUM_BARS =
-      2 * STAGES + 2 * NACC + 1 + 2 * RSTAGES + (CONV ? 2 * BSTAGES : 0);
+      2 * STAGES + 2 * NACC + 1 + 2 * RSTAGES + (CONV ? 2 * BSTAGES : 0) + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  // EPI_GS128: the tile's block scales; cluster split-K (rank 0 of a tile's
+  // cluster): the other ranks' partial sums, [csplit - 1][BM][BN] words
   static constexpr int OFF_SBLK = (OFF_MISC + 16 + 15) / 16 * 16;
-  static constexpr int smem_bytes(int kb_total) {
-    return 1024 + OFF_SBLK + (EPI == EPI_GS128 ? kb_total * SBLK_STRIDE * 4 : 0);
+  static constexpr int PART_BYTES = BM * BN * 4;
+  static constexpr int smem_bytes(int kb_total, int csplit = 0) {
+    return 1024 + OFF_SBLK + (EPI == EPI_GS128 ? kb_total * SBLK_STRIDE * 4 : 0) +
+           (csplit > 1 ? (csplit - 1) * PART_BYTES : 0);
   }
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N for M = 128");
   static_assert(EPI != EPI_GS128 || (I8 && !SWAP && BN % 64 == 0), "gs128 layout");
@@ -299,6 +305,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   uint64_t* raw_empty = raw_full + Cfg::RSTAGES;  // CONV: converters -> producer
   uint64_t* b_full = raw_empty + Cfg::RSTAGES;    // CONV: B producer -> MMA
   uint64_t* b_empty = b_full + Cfg::BSTAGES;      // CONV: MMA -> B producer
+  uint64_t* red_bar = b_empty + (Cfg::CONV ? Cfg::BSTAGES : 0);  // cluster split-K parts
   uint8_t* smRaw = smem + Cfg::OFF_RAW;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::OFF_MISC + 4);
@@ -330,6 +337,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         mbar_init(b_empty + s, 1);
       }
     }
+    // rank 0 of a split-K cluster: every epilogue thread of the other ranks
+    mbar_init(red_bar, (g.csplit > 1 ? g.csplit - 1 : 1) * NE * 32);
     *abort_flag = 0;
     *sk_flag = 0;
     fence_mbar_init();
@@ -340,6 +349,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   }
   tc_fence_before();
   __syncthreads();
+  // split-K clusters: the barriers of every rank are initialised before any
+  // rank arrives remotely
+  if (g.csplit > 1) cluster_sync();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   // a programmatic dependent of this grid may be scheduled now; it waits for
@@ -768,6 +780,49 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
             tmem_ld_acc<Cfg>(tb, c, nsub, v);
             store_chunk<Cfg>(g, rt, ct, rr, c, v, 0, scp);
           }
+        } else if (g.csplit > 1) {
+          // cluster split-K: the tile's K parts are the ranks of this cluster
+          // (rank r = part r); ranks > 0 write their sums into rank 0's shared
+          // memory and arrive on its barrier; rank 0 adds them in rank order
+          const uint32_t rank = cluster_ctarank();
+          uint32_t* red = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_SBLK);
+          if (rank != 0) {
+            const uint32_t dst = mapa_shared(
+                smem_u32(red + (static_cast<size_t>(rank - 1) * Cfg::BM + rr) * BN), 0);
+#pragma unroll 1
+            for (int c = 0; c < BN; c += CW) {
+              uint32_t v[CW];
+              tmem_ld_acc<Cfg>(tb, c, nsub, v);
+#pragma unroll
+              for (int j = 0; j < CW; j += 4)
+                st_cluster_v4(dst + (c + j) * 4, v[j], v[j + 1], v[j + 2], v[j + 3]);
+            }
+            mbar_arrive_cluster(mapa_shared(smem_u32(red_bar), 0));
+          } else if (wait_bounded_cluster(red_bar, 0, abort_flag)) {
+#pragma unroll 1
+            for (int c = 0; c < BN; c += CW) {
+              uint32_t v[CW];
+              tmem_ld_acc<Cfg>(tb, c, nsub, v);
+              for (int r = 1; r < g.csplit; ++r) {
+                const uint32_t* prow = red + (static_cast<size_t>(r - 1) * Cfg::BM + rr) * BN + c;
+#pragma unroll
+                for (int j = 0; j < CW; j += 4) {
+                  const uint4 w = *reinterpret_cast<const uint4*>(prow + j);
+                  const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                  for (int i = 0; i < 4; ++i) {
+                    uint32_t& acc = v[j + i];
+                    if constexpr (Cfg::I8)
+                      acc = static_cast<uint32_t>(static_cast<int32_t>(acc) +
+                                                  static_cast<int32_t>(wv[i]));
+                    else
+                      acc = __float_as_uint(__fadd_rn(__uint_as_float(acc), __uint_as_float(wv[i])));
+                  }
+                }
+              }
+              store_chunk<Cfg>(g, rt, ct, rr, c, v, 0, scp);
+            }
+          }
         } else {
           // stream-K part of a tile: publish, count, and the last arrival reduces
           const long long it0 = static_cast<long long>(s.tile) * g.kb_total;
@@ -853,6 +908,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
 
   tc_fence_before();
   __syncthreads();
+  // rank 0 keeps its shared memory until every rank's remote writes are done
+  if (g.csplit > 1) cluster_sync();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, Cfg::TMEM_COLS);

@@ -370,6 +370,38 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
                : "memory");
 }
+// 16 bytes to a shared-memory address of another CTA of the cluster.
+__device__ __forceinline__ void st_cluster_v4(uint32_t cluster_addr, uint32_t a, uint32_t b,
+                                              uint32_t c, uint32_t d) {
+  asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(cluster_addr), "r"(a),
+               "r"(b), "r"(c), "r"(d)
+               : "memory");
+}
+// wait_bounded with cluster-scope acquire: after it, this thread sees the
+// shared-memory writes that other CTAs of the cluster made before their
+// releasing arrivals on `bar`.
+__device__ __forceinline__ bool wait_bounded_cluster(uint64_t* bar, uint32_t parity,
+                                                     volatile int* abort_flag) {
+  const uint32_t a = smem_u32(bar);
+  const unsigned long long t0 = globaltimer_ns();
+  for (;;) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(a), "r"(parity), "r"(kSuspendHintNs)
+        : "memory");
+    if (ok) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      *abort_flag = 1;
+      atomicOr(&g_error_word, kErrTimeout);
+      return false;
+    }
+  }
+}
 // Pair TMA load: fills this CTA's shared memory; the transaction bytes are
 // counted on the mbarrier at `bar_cluster` (the pair leader's barrier).
 // `policy` is an L2 eviction-priority hint (createpolicy).

@@ -99,6 +99,7 @@ struct GemmPlan {
   int tiles_r, tiles_c;
   int kb_total;
   long long total_iters;
+  int csplit;       // > 1: whole splits combined inside a cluster of csplit CTAs
   size_t ws_bytes;  // counter region + stream-K slots (0: no workspace)
 };
 
@@ -136,6 +137,12 @@ GemmPlan plan_gemm(GemmKind kind, int64_t M, int64_t N, int64_t K, int sms) {
       // G = tiles * splits); long ranges use every SM instead
       const int splits = whole > p.kb_total ? p.kb_total : whole;
       p.grid = p.tiles_r * splits;
+      // W8A8: a tile's splits form one cluster and add their parts in
+      // distributed shared memory (rank 0 holds splits - 1 parts of
+      // 128 x bn words beside its operand ring)
+      const int max_split = p.bn == 16 ? 8 : 5;
+      if ((kind == GK_I8_SCALE || kind == GK_I8_I32) && splits >= 2 && splits <= max_split)
+        p.csplit = splits;
     } else {
       p.grid = sms;
     }
@@ -164,10 +171,45 @@ GemmPlan plan_gemm(GemmKind kind, int64_t M, int64_t N, int64_t K, int sms) {
   return p;
 }
 
+// Whether `clusters` clusters of `size` CTAs of this kernel can all be
+// resident at once (checked once per device, kernel and size).
 template <class Cfg>
-sq_status launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& g, int grid,
+bool clusters_fit(int size, int clusters, int smem) {
+  static std::atomic<int> cap[64][9];
+  int dev = 0;
+  if (size < 2 || size > 8 || cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+    return false;
+  int c = cap[dev][size].load(std::memory_order_acquire);
+  if (c == 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(size);
+    cfg.blockDim = dim3(Cfg::THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = size;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&c, gemm_kernel<Cfg>, &cfg) != cudaSuccess || c <= 0) {
+      cudaGetLastError();
+      c = -1;
+    }
+    cap[dev][size].store(c, std::memory_order_release);
+  }
+  return c >= clusters;
+}
+
+template <class Cfg>
+sq_status launch_gemm(const CUtensorMap& a, const CUtensorMap& b, GemmArgs g, int grid,
                       cudaStream_t st, bool pdl) {
-  const int smem = Cfg::smem_bytes(g.kb_total);
+  // cluster split-K needs room for the parts and every cluster resident at once;
+  // otherwise the tile's parts meet in the workspace
+  if (g.csplit > 1 && (Cfg::EPI == EPI_GS128 || Cfg::CONV ||
+                       Cfg::smem_bytes(g.kb_total, g.csplit) > 232448))
+    g.csplit = 0;
+  const int smem = Cfg::smem_bytes(g.kb_total, g.csplit);
   if (smem > 232448) return SQ_ERR_SHAPE;
   // Raise the kernel's dynamic shared-memory limit once per device (and only
   // upwards), so steady-state launches make no attribute call.
@@ -182,22 +224,38 @@ sq_status launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const GemmArgs
     while (cur < smem && !smem_set[dev].compare_exchange_weak(cur, smem)) {
     }
   }
-  if (!pdl) {
+  if (g.csplit > 1 && !clusters_fit<Cfg>(g.csplit, grid / g.csplit, smem)) {
+    g.csplit = 0;
+    return launch_gemm<Cfg>(a, b, g, grid, st, pdl);
+  }
+  if (!pdl && g.csplit <= 1) {
     gemm_kernel<Cfg><<<grid, Cfg::THREADS, smem, st>>>(a, b, g);
     return launch_status();
   }
   // programmatic dependent launch: the kernel may start while the preceding
-  // kernel on the stream runs; it requests only weights before griddep_wait
+  // kernel on the stream runs; it requests only weights before griddep_wait.
+  // Cluster split-K: the csplit CTAs of a tile are one cluster.
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(Cfg::THREADS);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  if (g.csplit > 1) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = g.csplit;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = na;
   if (cudaLaunchKernelEx(&cfg, gemm_kernel<Cfg>, a, b, g) != cudaSuccess) return SQ_ERR_CUDA;
   return launch_status();
 }
@@ -287,6 +345,7 @@ sq_status run_gemm(GemmKind kind, const void* act, const void* wt, const float* 
   g.ws_cnt = p.ws_bytes ? static_cast<unsigned int*>(ws) : nullptr;
   g.ws = p.ws_bytes ? reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + kCounterBytes)
                     : nullptr;
+  g.csplit = p.csplit;
 
   if (p.pair) {
     if (kind == GK_I8_SCALE) return launch_gemm2<Gemm2Cfg<EPI_SCALE, 6>>(ta, tb, g, st, pdl);
