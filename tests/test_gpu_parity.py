@@ -274,13 +274,14 @@ def test_fused_linear_pdl(M, N, K):
 
 # ------------------------------------------------ overlapped (PDL) launches
 
-@pytest.mark.parametrize("op", ["w8a8", "i32", "gs128", "w8a16"])
+@pytest.mark.parametrize("op", ["w8a8", "w8a8_cluster", "i32", "gs128", "w8a16"])
 def test_overlap_launch_policy(op):
     """sq_set_overlap(1): each GEMM is launched as a programmatic dependent of
     the call before it (weights requested before that call ends).  A chain of
     back-to-back calls on different weights gives exactly the results of
-    ordinary launches, and the first matches the oracle."""
-    M, N, K = (8, 1024, 2048) if op != "w8a16" else (16, 1024, 4096)
+    ordinary launches, and the first matches the oracle.  w8a8_cluster: a
+    shape whose K splits are combined inside clusters of 8 CTAs."""
+    M, N, K = {"w8a16": (16, 1024, 4096), "w8a8_cluster": (8, 2304, 4096)}.get(op, (8, 1024, 2048))
     x = inputs.gen_x(M, K, 23, inputs.XRecipe(col_count=3, col_factor=30.0))
     ws = [inputs.gen_w(N, K, 40 + i) for i in range(3)]
     q_a, s_tok = oracle.quant_per_token(x, None)
@@ -293,7 +294,7 @@ def test_overlap_launch_policy(op):
 
     def call(i):
         q_w, sc = qsd[i % 3]
-        if op == "w8a8":
+        if op in ("w8a8", "w8a8_cluster"):
             return sq.w8a8_scaled_mm(qad, std, q_w, sc)
         if op == "i32":
             return sq.w8a8_mm_i32(qad, q_w)
@@ -312,7 +313,7 @@ def test_overlap_launch_policy(op):
     for i in range(6):
         assert_same(over[i], plain[i].cpu(), f"{op} call {i}")
     q_w, sc = qs[0]
-    if op == "w8a8":
+    if op in ("w8a8", "w8a8_cluster"):
         assert_same(plain[0], oracle.w8a8_scaled_mm(q_a, s_tok, q_w, sc), "w8a8 vs oracle")
     elif op == "i32":
         assert_same(plain[0], oracle.mm_i32(q_a, q_w), "i32 vs oracle")
