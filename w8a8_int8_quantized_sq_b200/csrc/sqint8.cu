@@ -369,10 +369,8 @@ sq_status run_gemm(GemmKind kind, const void* act, const void* wt, const float* 
     case GK_GS128:
       return launch_gemm<GemmCfg<true, 128, 4, false, EPI_GS128>>(ta, tb, g, p.grid, st, pdl);
     case GK_BF16:
-      if (p.swap && p.bn == 16)
-        return launch_gemm<GemmCfg<false, 16, 8, true, EPI_SCALE>>(ta, tb, g, p.grid, st, pdl);
-      if (p.swap)
-        return launch_gemm<GemmCfg<false, 32, 8, true, EPI_SCALE>>(ta, tb, g, p.grid, st, pdl);
+      // bf16 weight copies exist only for M > 32 (no swapped schedule)
+      if (p.swap) return SQ_ERR_SHAPE;
       return launch_gemm<GemmCfg<false, 256, 4, false, EPI_SCALE>>(ta, tb, g, p.grid, st, pdl);
     case GK_W8A16_CONV:
       if (p.bn == 16)
