@@ -169,6 +169,32 @@ sq_status sq_quant_weight(const void* w_bf16, const float* smooth, int8_t* q_w, 
  * own quantisation kernel.  Always returns SQ_OK. */
 sq_status sq_set_overlap(int enable);
 
+/* The schedule one GEMM call would use on a device with `sms` streaming
+ * multiprocessors, worked out on the host alone (no GPU needed; the pages
+ * have no counterpart: it describes this library's kernels).  op: SQ_OP_*.
+ * kernel: 0 = CTA pairs (256 x 256 output tiles), 1 = one CTA per tile,
+ * 2 = swapped small-M tiles on stream-K ranges (partial tiles meet in the
+ * workspace), 3 = swapped small-M tiles whose K parts meet inside a
+ * thread-block cluster (a call falls back to 2 when the device cannot hold
+ * every cluster at once or the parts do not fit in shared memory).
+ * tile_m x tile_n: tokens x output channels per tile.  grid: CTAs (for
+ * kernel 0 an upper bound: the launch takes the active-cluster limit).
+ * splits: K parts per tile when every CTA owns one part of one tile, 0 when
+ * the stream-K ranges cross tiles, 1 for whole-K tiles.  workspace_bytes: as
+ * sq_workspace_bytes.  Returns SQ_ERR_SHAPE for sms <= 0 or a bad shape or op,
+ * SQ_ERR_NULL for out == NULL. */
+typedef struct {
+  int32_t kernel;
+  int32_t grid;
+  int32_t tile_m;
+  int32_t tile_n;
+  int32_t splits;
+  uint64_t workspace_bytes;
+} sq_plan_info;
+
+sq_status sq_describe_plan(int op, int64_t M, int64_t N, int64_t K, int sms,
+                           sq_plan_info* out);
+
 /* Diagnostics ------------------------------------------------------------ */
 
 /* Synchronises the current device, then returns SQ_ERR_TIMEOUT if any kernel

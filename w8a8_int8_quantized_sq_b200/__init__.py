@@ -66,6 +66,7 @@ def lib() -> ctypes.CDLL:
                 "sq_quant_weight": [vp, vp, vp, vp, i64, i64, i64, vp],
                 "sq_check_device_error": [ctypes.c_int],
                 "sq_set_overlap": [ctypes.c_int],
+                "sq_describe_plan": [ctypes.c_int, i64, i64, i64, ctypes.c_int, vp],
             }
             for name, args in sig.items():
                 f = getattr(L, name)
@@ -82,7 +83,7 @@ def lib() -> ctypes.CDLL:
 EXPORTS = ("sq_quant_per_token", "w8a8_scaled_mm", "w8a8_gs128_mm", "w8a16_mm",
            "sq_workspace_bytes", "w8a8_mm_i32", "sq_smooth_factors", "sq_quant_weight",
            "sq_check_device_error", "sq_status_string", "w8a8_scaled_mm_noalloc",
-           "sq_w8a8_linear", "sq_set_overlap")
+           "sq_w8a8_linear", "sq_set_overlap", "sq_describe_plan")
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -224,6 +225,22 @@ def quant_weight(w, smooth: Optional[torch.Tensor] = None, group: int = 0):
     _check("sq_quant_weight", lib().sq_quant_weight(
         _ptr(w), _ptr(smooth), _ptr(q), _ptr(sc), N, K, group, _stream(w.device)))
     return q, sc
+
+
+class PlanInfo(ctypes.Structure):
+    """sq_plan_info (include/sqint8.h)."""
+    _fields_ = [("kernel", ctypes.c_int32), ("grid", ctypes.c_int32), ("tile_m", ctypes.c_int32),
+                ("tile_n", ctypes.c_int32), ("splits", ctypes.c_int32),
+                ("workspace_bytes", ctypes.c_uint64)]
+
+
+def describe_plan(op: int, M: int, N: int, K: int, sms: int) -> dict:
+    """The schedule a GEMM call would use on a device with `sms` SMs
+    (sq_describe_plan; host only, no GPU needed)."""
+    L = lib()
+    info = PlanInfo()
+    _check("sq_describe_plan", L.sq_describe_plan(op, M, N, K, sms, ctypes.byref(info)))
+    return {name: getattr(info, name) for name, _ in PlanInfo._fields_}
 
 
 def set_overlap(enable: bool) -> None:

@@ -99,6 +99,7 @@ struct GemmPlan {
   int tiles_r, tiles_c;
   int kb_total;
   long long total_iters;
+  int splits;       // swapped: K parts per tile with whole splits, 0 for stream-K ranges
   int csplit;       // > 1: whole splits combined inside a cluster of csplit CTAs
   size_t ws_bytes;  // counter region + stream-K slots (0: no workspace)
 };
@@ -137,6 +138,7 @@ GemmPlan plan_gemm(GemmKind kind, int64_t M, int64_t N, int64_t K, int sms) {
       // G = tiles * splits); long ranges use every SM instead
       const int splits = whole > p.kb_total ? p.kb_total : whole;
       p.grid = p.tiles_r * splits;
+      p.splits = splits;
       // W8A8: a tile's splits form one cluster and add their parts in
       // distributed shared memory (rank 0 holds splits - 1 parts of
       // 128 x bn words beside its operand ring)
@@ -556,6 +558,47 @@ size_t sq_workspace_bytes(int op, int64_t M, int64_t N, int64_t K) {
     case SQ_OP_W8A16: return w8a16_ws_bytes(M, N, K, sms, nullptr);
   }
   return 0;
+}
+
+sq_status sq_describe_plan(int op, int64_t M, int64_t N, int64_t K, int sms,
+                           sq_plan_info* out) {
+  if (!out) return SQ_ERR_NULL;
+  const sq_status s = check_mnk(M, N, K);
+  if (s != SQ_OK) return s;
+  if (sms <= 0) return SQ_ERR_SHAPE;
+  GemmKind kind;
+  switch (op) {
+    case SQ_OP_W8A8: kind = GK_I8_SCALE; break;
+    case SQ_OP_W8A8_I32: kind = GK_I8_I32; break;
+    case SQ_OP_GS128: kind = GK_GS128; break;
+    case SQ_OP_W8A16: kind = M <= 32 ? GK_W8A16_CONV : GK_BF16; break;
+    default: return SQ_ERR_SHAPE;
+  }
+  const GemmPlan p = plan_gemm(kind, M, N, K, sms);
+  const int tiles = p.tiles_r * p.tiles_c;
+  sq_plan_info r{};
+  if (p.pair) {
+    r.kernel = 0;
+    r.grid = 2 * (tiles < sms / 2 ? tiles : sms / 2);
+    r.tile_m = 256;
+    r.tile_n = 256;
+    r.splits = 1;
+  } else if (!p.swap) {
+    r.kernel = 1;
+    r.grid = p.grid;
+    r.tile_m = 128;
+    r.tile_n = p.bn;
+    r.splits = 1;
+  } else {
+    r.kernel = p.csplit > 1 ? 3 : 2;
+    r.grid = p.grid;
+    r.tile_m = p.bn;
+    r.tile_n = 128;
+    r.splits = p.splits;
+  }
+  r.workspace_bytes = op == SQ_OP_W8A16 ? w8a16_ws_bytes(M, N, K, sms, nullptr) : p.ws_bytes;
+  *out = r;
+  return SQ_OK;
 }
 
 sq_status w8a8_scaled_mm(const int8_t* q_a, const float* s_tok, const int8_t* q_w,
