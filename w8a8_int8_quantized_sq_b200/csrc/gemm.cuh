@@ -3,9 +3,10 @@
 //   warp 0      : TMA producer (one elected thread) filling a ring of
 //                 shared-memory stages, each one 128-byte-wide K block of
 //                 A (128 rows) and B (BN rows), 128-byte swizzled.
-//   warp 1      : allocates tensor memory; one thread issues tcgen05.mma
-//                 (kind::i8 with int32 accumulators, or kind::f16 with BF16
-//                 operands and fp32 accumulators) into TMEM.
+//   warp 1      : allocates tensor memory; the whole warp runs the issue
+//                 loop and one elected lane issues tcgen05.mma (kind::i8
+//                 with int32 accumulators, or kind::f16 with BF16 operands
+//                 and fp32 accumulators) into TMEM.
 //   warps 2..   : epilogue; tcgen05.ld of the accumulators, scale, convert,
 //                 store.  Double-buffered accumulators let the epilogue of
 //                 one tile overlap the mainloop of the next.
@@ -21,6 +22,9 @@
 // finish its part: every part is written to a per-CTA slot of the
 // workspace, an atomic counter per tile elects the last arrival, which sums
 // the parts in CTA order and runs the epilogue, then resets the counter.
+// When every CTA owns one K part of one tile (csplit > 1), a tile's CTAs are
+// one thread-block cluster instead and the parts meet in rank 0's shared
+// memory.
 //
 // EPI_GS128 (group-size-128 weight scales): every 128-wide K block is MMA'd
 // into a fresh int32 TMEM buffer (4 in rotation).  The epilogue warps load a
@@ -473,7 +477,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           // its box row, 16-byte chunk j at position j ^ (row & 7).  This
           // thread converts chunks 2*half, 2*half+1 (32 codes -> 32 bf16, two
           // per column, lower K in the low half) into TMEM columns 16*half ..
-          // 16*half+15 of the K block's A slot.
+          // 16*half+15 of the K block's part of the A stage.
           auto chunk = [&](int c, int jj) {
             return *reinterpret_cast<const uint4*>(
                 raw + (c >> 1) * Cfg::RAW_BOX_BYTES + row * 128 +
