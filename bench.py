@@ -182,6 +182,34 @@ def dist_info():
     return ws, rank, local
 
 
+def replica_collectives(world: int, dev: torch.device):
+    """The only collectives of the replicas: a barrier (plus a device
+    synchronize on CUDA) and the maximum of a per-rank time.  Any backend:
+    NCCL on the GPUs, gloo in the CPU tests."""
+    import torch.distributed as dist
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        if dev.type == "cuda":
+            torch.cuda.synchronize(dev)
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    return barrier, max_over_ranks
+
+
+def whole_job_tops(ops_per_step: float, steps: int, world: int, seconds: float) -> float:
+    """Every replica runs `steps` steps; the job's rate is all ranks' work
+    over the slowest rank's time."""
+    return ops_per_step * steps * world / seconds / 1e12
+
+
 # ------------------------------------------------------------ CPU oracle leg
 def oracle_sample(wl, target_s: float, max_rows: int = None):
     """Times the CPU oracle (quant + W8A8 GEMM) on a bounded row sample."""
@@ -273,17 +301,7 @@ def main():
     torch.cuda.set_device(dev)
     sq.lib()  # fails loudly if the CUDA library is missing
 
-    def barrier():
-        if world > 1:
-            torch.distributed.barrier()
-        torch.cuda.synchronize()
-
-    def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        return float(t.item())
+    barrier, max_over_ranks = replica_collectives(world, dev)
 
     # ---------------- prefill W8A8 (the headline workload)
     wl = inputs.workload(2)
@@ -339,7 +357,7 @@ def main():
     quant_s = time_graph(lambda i: sq.quant_per_token(xs[i % 3], inv_s), 12, reps=3)
     del xs
     ops_step = 2.0 * M * N * K
-    value = ops_step * args.steps * world / total_s / 1e12
+    value = whole_job_tops(ops_step, args.steps, world, total_s)
     int8_peak = peaks["bf16_tflops"] * INT8_PER_BF16
     gemm_tops = ops_step / gemm_s / 1e12
 
@@ -364,7 +382,7 @@ def main():
     b.record()
     barrier()
     e2e_s = max_over_ranks(a.elapsed_time(b) * 1e-3)
-    e2e = {"value": ops_step * e2e_steps * world / e2e_s / 1e12, "unit": "TOPS",
+    e2e = {"value": whole_job_tops(ops_step, e2e_steps, world, e2e_s), "unit": "TOPS",
            "h2d_bytes_per_step": x_h.numel() * 2, "d2h_bytes_per_step": y_h.numel() * 2,
            "steps": e2e_steps}
     del x_h, y_h, x_d
