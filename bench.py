@@ -241,7 +241,10 @@ def reference_arm(args, peaks):
         return 0
     from w8a8_int8_quantized_sq_b200 import inputs
     wl = inputs.workload(2)
-    rows, nt, run = oracle_sample(wl, target_s=0.5)
+    # about 0.5 s of oracle work per step, less for long runs: the whole
+    # --steps + --warmup run stays near two minutes
+    per_step = min(0.5, 120.0 / (args.steps + args.warmup))
+    rows, nt, run = oracle_sample(wl, target_s=per_step)
     ops_step = 2.0 * rows * wl.N * wl.K
     for _ in range(args.warmup):
         run(rows)
