@@ -56,6 +56,7 @@ struct GemmArgs {
   unsigned int* ws_cnt;   // stream-K arrival counters [num_tiles]
   int csplit;             // > 1: the csplit CTAs of a tile form a cluster and
                           // combine their K parts in distributed shared memory
+  int pdl;                // launched as a programmatic dependent
 };
 
 __host__ __device__ constexpr int pow2_at_least(int v) {
@@ -530,11 +531,13 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       it.init(g);
       Seg s;
       bool ok = true;
-      // The weight operand (A when SWAP, else B) of the first STAGES fills is
-      // requested before griddep_wait, so that under a programmatic launch the
-      // weight stream starts while the preceding kernel still produces the
-      // activations; their activation tiles follow right after the wait.
-      bool waited = false;
+      // Under a programmatic launch the weight operand (A when SWAP, else B)
+      // of the first STAGES fills is requested before griddep_wait, so that
+      // the weight stream starts while the preceding kernel still produces
+      // the activations; their activation tiles follow right after the wait.
+      // Otherwise every fill requests both at once (so the first stage is
+      // not queued behind STAGES weight tiles).
+      bool waited = g.pdl == 0;
       int pend_kb[STAGES], pend_row[STAGES];
       auto act_load = [&](int st, int kb, int row) {
         if constexpr (Cfg::SWAP)

@@ -206,6 +206,7 @@ bool clusters_fit(int size, int clusters, int smem) {
 template <class Cfg>
 sq_status launch_gemm(const CUtensorMap& a, const CUtensorMap& b, GemmArgs g, int grid,
                       cudaStream_t st, bool pdl) {
+  g.pdl = pdl ? 1 : 0;
   // cluster split-K needs room for the parts and every cluster resident at once;
   // otherwise the tile's parts meet in the workspace
   if (g.csplit > 1 && (Cfg::EPI == EPI_GS128 || Cfg::CONV ||
