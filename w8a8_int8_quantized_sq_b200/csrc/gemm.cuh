@@ -93,7 +93,7 @@ struct GemmCfg {
   static constexpr int A_BYTES = BM * KB_BYTES;
   static constexpr int B_BYTES = BN * KB_BYTES;
   // raw stage: RK K blocks of int8 weight rows, as RK/2 boxes of 128 rows x
-  // 128 bytes (two K blocks per row, 128-byte swizzle), then the RK B tiles
+  // 128 bytes (two K blocks per row, 128-byte swizzle)
   static constexpr int RK = 4;
   static constexpr int RAW_BOX_BYTES = BM * 128;
   static constexpr int RAW_A_BYTES = (RK / 2) * RAW_BOX_BYTES;
