@@ -142,23 +142,29 @@ def test_w8a8_scaled_mm_configs(cfg):
     assert_same(y3, ref, "y (repeat)")
 
 
-def test_w8a8_prefill_full_size_sampled_rows():
-    """M=8192, K=5120, N=34816: the whole GEMM on the GPU, oracle on sampled rows."""
+def test_w8a8_prefill_full_size():
+    """M=8192, K=5120, N=34816, every output: the int32 accumulators of the
+    mainloop and y of the benchmarked fused layer (sq_w8a8_linear) and of
+    w8a8_scaled_mm, each against the oracle, 1024 token rows at a time."""
     d = workload(2)
     c = to_cuda(d)
     q_a, s_tok = sq.quant_per_token(c["x"], c["inv_s"])
     assert_same(q_a, d["q_a"], "q_a")
     assert_same(s_tok, d["s_tok"], "s_tok")
-    y = sq.w8a8_scaled_mm(c["q_a"], c["s_tok"], c["q_w"], c["s_ch"])
-    rows = sorted({0, 1, 2, 3, 4, 127, 128, 511, 512, 515, 4096, 8191} |
-                  set(np.random.default_rng(0).integers(0, 8192, 12).tolist()))
-    ref = oracle.w8a8_scaled_mm(d["q_a"], d["s_tok"], d["q_w"], d["s_ch"], rows=rows)
-    assert_same(y.cpu()[rows], ref, "y sampled rows")
-    # a column sample over every row too (catches errors in other row tiles)
-    cols = [0, 255, 256, 17407, 34815]
-    acc = oracle.mm_i32(d["q_a"], d["q_w"][cols].contiguous())
-    yc = oracle.epilogue_ch(acc, d["s_tok"], d["s_ch"][cols].contiguous())
-    assert_same(y.cpu()[:, cols].contiguous(), yc, "y sampled columns")
+    del q_a, s_tok
+    acc = sq.w8a8_mm_i32(c["q_a"], c["q_w"]).cpu()
+    y_lin = sq.linear_w8a8(c["x"], c["inv_s"], c["q_w"], c["s_ch"]).cpu()
+    y_mm = sq.w8a8_scaled_mm(c["q_a"], c["s_tok"], c["q_w"], c["s_ch"]).cpu()
+    del c
+    torch.cuda.empty_cache()
+    M = d["q_a"].shape[0]
+    for r0 in range(0, M, 1024):
+        rows = list(range(r0, min(M, r0 + 1024)))
+        acc_ref = oracle.mm_i32(d["q_a"], d["q_w"], rows=rows)
+        assert_same(acc[r0:r0 + len(rows)], acc_ref, f"int32 acc rows {r0}..")
+        y_ref = oracle.epilogue_ch(acc_ref, d["s_tok"][r0:r0 + len(rows)].contiguous(), d["s_ch"])
+        assert_same(y_lin[r0:r0 + len(rows)], y_ref, f"y (sq_w8a8_linear) rows {r0}..")
+        assert_same(y_mm[r0:r0 + len(rows)], y_ref, f"y (w8a8_scaled_mm) rows {r0}..")
 
 
 # ---------------------------------------------------------------- gs128
@@ -196,7 +202,13 @@ def _check_w8a16(x, q_w, s_ch, rows=None):
     diff = (y.double() - ref.double()).abs()
     ulp = bf16_ulp(ref)
     assert torch.all(diff <= ulp + gamma * mag), float((diff - ulp - gamma * mag).max())
-    within_1ulp = float((diff <= ulp).double().mean())
+    beyond = int((diff > ulp).sum())
+    within_1ulp = 1.0 - beyond / diff.numel()
+    # the count of outputs that need the accumulation-order clause (printed
+    # with -s; the bar above holds for every output)
+    print(f"\nW8A16 M={x.shape[0]} K={K} N={q_w.shape[0]}"
+          f"{'' if rows is None else f' ({len(rows)} rows)'}: {beyond} of {diff.numel()} "
+          f"outputs beyond 1 bf16 ulp, max excess {float((diff / ulp).max()):.3f} ulp")
     assert within_1ulp > 0.999, within_1ulp
     return within_1ulp
 
@@ -207,9 +219,13 @@ def test_w8a16_decode(M):
     _check_w8a16(d["x"], d["q_w"], d["s_ch"])
 
 
-def test_w8a16_prefill_sampled_rows():
+def test_w8a16_prefill_every_row_tile():
+    """M=8192 (bf16 copy + BF16 pair GEMM): one seeded row in every 128-row
+    tile, plus the rows at the edges of the x50 outlier windows."""
     d = workload(4, 8192)
-    rows = [0, 1, 511, 512, 513, 4095, 8191]
+    rng = np.random.default_rng(8192)
+    rows = sorted({0, 1, 511, 512, 513, 4095, 8191} |
+                  {t * 128 + int(rng.integers(0, 128)) for t in range(8192 // 128)})
     _check_w8a16(d["x"], d["q_w"], d["s_ch"], rows=rows)
 
 

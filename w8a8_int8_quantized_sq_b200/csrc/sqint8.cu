@@ -1,6 +1,7 @@
 // sqint8.cu -- host side of the C ABI declared in include/sqint8.h:
 // argument checks, launch planning, tensor-map encoding and kernel launches.
-// The library holds no device memory of its own except one error word.
+// The library's own device memory is one error word plus the fixed scratch
+// array of w8a8_scaled_mm_noalloc (end of this file); nothing else.
 #include <atomic>
 #include <cstdlib>
 #include <mutex>
