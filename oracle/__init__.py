@@ -40,9 +40,30 @@ def lib() -> ctypes.CDLL:
         L.oracle_w8a8_scaled_mm.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, i64, vp]
         L.oracle_gs128_mm.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, i64, vp]
         L.oracle_w8a16_mm.argtypes = [vp, vp, vp, i64, i64, i64, vp, i64, vp, vp]
+        flt, i32 = ctypes.c_float, ctypes.c_int
+        L.oracle_fold_norm_weight.argtypes = [vp, i64, i32, vp, vp]
+        L.oracle_sumsq_f32.argtypes = [vp, i64]
+        L.oracle_sumsq_f32.restype = ctypes.c_float
+        L.oracle_rmsnorm_quant.argtypes = [vp, i64, i64, vp, flt, i64, vp, vp, vp, vp]
+        L.oracle_quant_per_group.argtypes = [vp, i64, i64, vp, vp, vp]
+        L.oracle_pg128_mm.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, i64, vp]
+        L.oracle_dequant_weight_group.argtypes = [vp, vp, i64, i64, vp]
+        L.oracle_w8a16_group_mm.argtypes = [vp, vp, vp, i64, i64, i64, vp, i64, vp, vp]
+        L.oracle_f32_to_e4m3.argtypes = [flt]
+        L.oracle_f32_to_e4m3.restype = ctypes.c_uint8
+        L.oracle_e4m3_to_f32.argtypes = [ctypes.c_uint8]
+        L.oracle_e4m3_to_f32.restype = flt
+        L.oracle_quant_fp8_per_group.argtypes = [vp, i64, i64, vp, vp, vp]
+        L.oracle_quant_fp8_block.argtypes = [vp, i64, i64, vp, vp, vp]
+        L.oracle_fp8_block_mm.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, i64, vp, vp]
         for name in ("oracle_smooth_factors", "oracle_fold_weight", "oracle_quant_weight",
                      "oracle_quant_per_token", "oracle_mm_i32", "oracle_epilogue_ch",
-                     "oracle_w8a8_scaled_mm", "oracle_gs128_mm", "oracle_w8a16_mm"):
+                     "oracle_w8a8_scaled_mm", "oracle_gs128_mm", "oracle_w8a16_mm",
+                     "oracle_fold_norm_weight", "oracle_rmsnorm_quant",
+                     "oracle_quant_per_group", "oracle_pg128_mm",
+                     "oracle_dequant_weight_group", "oracle_w8a16_group_mm",
+                     "oracle_quant_fp8_per_group", "oracle_quant_fp8_block",
+                     "oracle_fp8_block_mm"):
             getattr(L, name).restype = ctypes.c_int
     return _lib
 
@@ -167,4 +188,116 @@ def w8a16_mm(x, q_w, s_ch, rows=None, with_bound: bool = False):
     mag = torch.empty((nr, N), dtype=torch.float64) if with_bound else None
     _check(lib().oracle_w8a16_mm(_p(x.contiguous()), _p(q_w), _p(s_ch), M, N, K, _p(r), nr,
                                  _p(y), _p(mag)), "w8a16_mm")
+    return (y, mag) if with_bound else y
+
+
+# ------------------------------------------------------------ next rows
+
+def fold_norm_weight(w_norm: torch.Tensor, inv_s: Optional[torch.Tensor],
+                     zero_centered: bool = True) -> torch.Tensor:
+    """gamma fp32 [K] = (1 + w or w) * inv_s: the norm weight with 1/s folded in."""
+    K = w_norm.numel()
+    g = torch.empty(K, dtype=torch.float32)
+    _check(lib().oracle_fold_norm_weight(_p(w_norm.contiguous()), K, 1 if zero_centered else 0,
+                                         _p(inv_s), _p(g)), "fold_norm_weight")
+    return g
+
+
+def sumsq_f32(h: torch.Tensor) -> float:
+    """Exact sum of squares of a bf16 vector, rounded once to fp32."""
+    h = h.contiguous()
+    return lib().oracle_sumsq_f32(_p(h), h.numel())
+
+
+def rmsnorm_quant(h: torch.Tensor, gamma: torch.Tensor, eps: float, group: int = 0,
+                  r_in: Optional[torch.Tensor] = None):
+    """(q int8 [M,K], scales fp32 [M] or [M, K/128], r fp32 [M]); group 0 = per token."""
+    M, K = h.shape
+    g = K if group == 0 else group
+    q = torch.empty((M, K), dtype=torch.int8)
+    sc = torch.empty((M,) if g == K else (M, K // g), dtype=torch.float32)
+    r = torch.empty(M, dtype=torch.float32)
+    _check(lib().oracle_rmsnorm_quant(_p(h.contiguous()), M, K, _p(gamma.contiguous()), eps, g,
+                                      _p(r_in), _p(q), _p(sc), _p(r)), "rmsnorm_quant")
+    return q, sc, r
+
+
+def quant_per_group(x: torch.Tensor, inv_s: Optional[torch.Tensor] = None):
+    """(q int8 [M,K], s_a fp32 [M, K/128])."""
+    M, K = x.shape
+    q = torch.empty((M, K), dtype=torch.int8)
+    s = torch.empty((M, K // 128), dtype=torch.float32)
+    _check(lib().oracle_quant_per_group(_p(x.contiguous()), M, K, _p(inv_s), _p(q), _p(s)),
+           "quant_per_group")
+    return q, s
+
+
+def pg128_mm(q_a, s_a, q_w, s_blk, rows=None) -> torch.Tensor:
+    M, K = q_a.shape
+    N = q_w.shape[0]
+    r, nr = _rows(rows, M)
+    y = torch.empty((nr, N), dtype=torch.bfloat16)
+    _check(lib().oracle_pg128_mm(_p(q_a), _p(s_a.contiguous()), _p(q_w), _p(s_blk.contiguous()),
+                                 M, N, K, _p(r), nr, _p(y)), "pg128_mm")
+    return y
+
+
+def dequant_weight_group(q_w: torch.Tensor, s_grp: torch.Tensor) -> torch.Tensor:
+    N, K = q_w.shape
+    w = torch.empty((N, K), dtype=torch.bfloat16)
+    _check(lib().oracle_dequant_weight_group(_p(q_w), _p(s_grp.contiguous()), N, K, _p(w)),
+           "dequant_weight_group")
+    return w
+
+
+def w8a16_group_mm(x, q_w, s_grp, rows=None, with_bound: bool = False):
+    """y bf16 [rows, N]; with_bound also returns sum|x w_hat| (fp64)."""
+    M, K = x.shape
+    N = q_w.shape[0]
+    r, nr = _rows(rows, M)
+    y = torch.empty((nr, N), dtype=torch.bfloat16)
+    mag = torch.empty((nr, N), dtype=torch.float64) if with_bound else None
+    _check(lib().oracle_w8a16_group_mm(_p(x.contiguous()), _p(q_w), _p(s_grp.contiguous()),
+                                       M, N, K, _p(r), nr, _p(y), _p(mag)), "w8a16_group_mm")
+    return (y, mag) if with_bound else y
+
+
+def f32_to_e4m3_bits(v: float) -> int:
+    return lib().oracle_f32_to_e4m3(v)
+
+
+def e4m3_bits_to_f32(b: int) -> float:
+    return lib().oracle_e4m3_to_f32(b)
+
+
+def quant_fp8_per_group(x: torch.Tensor, inv_s: Optional[torch.Tensor] = None):
+    """(q e4m3 bits uint8 [M,K], s_a fp32 [M, K/128])."""
+    M, K = x.shape
+    q = torch.empty((M, K), dtype=torch.uint8)
+    s = torch.empty((M, K // 128), dtype=torch.float32)
+    _check(lib().oracle_quant_fp8_per_group(_p(x.contiguous()), M, K, _p(inv_s), _p(q), _p(s)),
+           "quant_fp8_per_group")
+    return q, s
+
+
+def quant_fp8_block(w: torch.Tensor, smooth: Optional[torch.Tensor] = None):
+    """(q e4m3 bits uint8 [N,K], s_w fp32 [N/128, K/128])."""
+    N, K = w.shape
+    q = torch.empty((N, K), dtype=torch.uint8)
+    s = torch.empty((N // 128, K // 128), dtype=torch.float32)
+    _check(lib().oracle_quant_fp8_block(_p(w.contiguous()), N, K, _p(smooth), _p(q), _p(s)),
+           "quant_fp8_block")
+    return q, s
+
+
+def fp8_block_mm(q_a, s_a, q_w, s_w, rows=None, with_bound: bool = False):
+    """y bf16 [rows, N]; with_bound also returns sum_kb |scale| sum|a w| (fp64)."""
+    M, K = q_a.shape
+    N = q_w.shape[0]
+    r, nr = _rows(rows, M)
+    y = torch.empty((nr, N), dtype=torch.bfloat16)
+    mag = torch.empty((nr, N), dtype=torch.float64) if with_bound else None
+    _check(lib().oracle_fp8_block_mm(_p(q_a.contiguous()), _p(s_a.contiguous()),
+                                     _p(q_w.contiguous()), _p(s_w.contiguous()), M, N, K,
+                                     _p(r), nr, _p(y), _p(mag)), "fp8_block_mm")
     return (y, mag) if with_bound else y
