@@ -27,7 +27,12 @@
  *       INT8 weights, dynamic per-token INT8 activations.
  *  [P5] "Qwen3.8-27B-GPTQ-INT8-W8A8-GS128", "Quantization details" and
  *       "Why group_size 128": one weight scale per 128-wide K block with INT8
- *       x INT8 compute and dynamically quantised inputs.
+ *       x INT8 compute and dynamically quantised inputs; "Serving (vLLM,
+ *       gfx908 fork)": fused RMSNorm with per-group INT8 quantised output and
+ *       W8A8 INT8 GEMMs at every M.
+ *  [P3b] "Qwen3.8-27B - FP8 block + AWQ", "Recipe" item 2 and the note after
+ *       it: FP8 weights with one scale per [128, 128] block, activations
+ *       quantised dynamically per group, quantised dimensions divisible by 128.
  */
 #ifndef SQINT8_H
 #define SQINT8_H
@@ -49,7 +54,8 @@ typedef enum {
 } sq_status;
 
 /* Operation ids for sq_workspace_bytes. */
-enum { SQ_OP_W8A8 = 0, SQ_OP_GS128 = 1, SQ_OP_W8A16 = 2, SQ_OP_W8A8_I32 = 3 };
+enum { SQ_OP_W8A8 = 0, SQ_OP_GS128 = 1, SQ_OP_W8A16 = 2, SQ_OP_W8A8_I32 = 3,
+       SQ_OP_PG128 = 4, SQ_OP_FP8BLK = 5, SQ_OP_W8A16_GROUP = 6 };
 
 /* Per-token dynamic INT8 quantisation with the SmoothQuant 1/s fold [P1, P3, P4].
  * For each row m of x (BF16 [M,K]):  x'[k] = f32(x[m,k]) * inv_smooth[k]
@@ -127,6 +133,82 @@ sq_status w8a16_mm(const void* x_bf16, const int8_t* q_w, const float* s_ch, voi
 sq_status w8a8_scaled_mm_noalloc(const int8_t* q_a, const float* s_tok, const int8_t* q_w,
                                  const float* s_ch, void* y_bf16, int64_t M, int64_t N,
                                  int64_t K, void* stream);
+
+/* Next rows of the layer ----------------------------------------------- */
+
+/* Norm weight with the SmoothQuant factor folded in [P1 "Recipe" item 1:
+ * zero-centred norms absorb 1/s; P3 "Recipe" item 1]: gamma fp32 [K],
+ * gamma[k] = f32(g_k * inv_smooth[k]) with g_k = 1 + f32(w_norm[k]) when
+ * zero_centered != 0, else f32(w_norm[k]); inv_smooth may be NULL (= 1).
+ * w_norm_bf16: BF16 [K]. */
+sq_status sq_fold_norm_weight(const void* w_norm_bf16, int zero_centered,
+                              const float* inv_smooth, float* gamma, int64_t K, void* stream);
+
+/* Fused RMSNorm + SmoothQuant fold + dynamic INT8 quantisation [P1 "Recipe"
+ * items 1-2, P5 "Serving": RMSNorm with per-group INT8 quantised output].
+ * Per row m of h (BF16 [M,K]): ss = sum_k f32(h)^2 rounded once to fp32
+ * (accumulated in fp64); r = 1 / sqrt(ss / K + eps) (IEEE fp32 division,
+ * addition and square root); x'_k = (f32(h_k) * r) * gamma[k] (two fp32
+ * roundings; gamma from sq_fold_norm_weight); then the quantisation of
+ * sq_quant_per_token over the row (group == 0 or K: scales fp32 [M]) or over
+ * each 128-column block (group == 128: scales fp32 [M, K/128]).  inv_rms
+ * (fp32 [M], may be NULL) receives r.  eps > 0; K <= 24576.  The fp64 sum
+ * of squares rounds to the exact sum's fp32 value except when that sum lies
+ * within about K * 2^-53 (relative) of a point halfway between two fp32
+ * numbers. */
+sq_status sq_rmsnorm_quant(const void* h_bf16, const float* gamma, float eps, int64_t group,
+                           int8_t* q_i8, float* scales, float* inv_rms, int64_t M, int64_t K,
+                           void* stream);
+
+/* Per-group (1 x 128) dynamic INT8 activation quantisation with the 1/s fold
+ * [P5 "Serving": per-group INT8 quant-out]: sq_quant_per_token's arithmetic on
+ * every 128-wide block of every row; s_a fp32 [M, K/128]. */
+sq_status sq_quant_per_group(const void* x_bf16, const float* inv_smooth, int8_t* q_i8,
+                             float* s_a, int64_t M, int64_t K, void* stream);
+
+/* Per-group activations x gs128 weights [P5 "Why group_size 128", "Serving"]:
+ * with P_kb the exact int32 partial over K block kb, acc = 0; for kb
+ * ascending: acc = fmaf(f32(P_kb), f32(s_a[m,kb] * s_blk[n,kb]), acc);
+ * y = bf16_rne(acc).  q_a int8 [M,K], s_a fp32 [M, K/128], q_w int8 [N,K],
+ * s_blk fp32 [N, K/128] (sq_quant_weight with group 128).  Workspace as
+ * for w8a8_scaled_mm (SQ_OP_PG128; currently always 0). */
+sq_status w8a8_pg128_mm(const int8_t* q_a, const float* s_a, const int8_t* q_w,
+                        const float* s_blk, void* y_bf16, int64_t M, int64_t N, int64_t K,
+                        void* workspace, size_t ws_bytes, void* stream);
+
+/* Group-wise W8A16 [P2 "Why W8A16 on Ampere": weight-only kernels
+ * reconstruct 16-bit weights; eight integer bits with group-wise scaling]:
+ * w_hat[n,k] = bf16_rne(f32(q_w[n,k] * s_grp[n, k/128])) (codes and scales
+ * from sq_quant_weight with group 128), y = bf16_rne(sum_k x[m,k] *
+ * w_hat[n,k]) with exact products accumulated in fp32 (the order of the
+ * fp32 sum is the kernel's).  Workspace as for w8a16_mm (SQ_OP_W8A16_GROUP). */
+sq_status w8a16_group_mm(const void* x_bf16, const int8_t* q_w, const float* s_grp,
+                         void* y_bf16, int64_t M, int64_t N, int64_t K, void* workspace,
+                         size_t ws_bytes, void* stream);
+
+/* FP8 (OCP E4M3: bias 7, largest finite 448) per-group activations [P3b]:
+ * per 128-wide block of each row, v = f32(x) * inv_smooth[k] (inv_smooth may
+ * be NULL), amax = max|v|, s_a = amax / 448, code = e4m3_rne_satfinite(v *
+ * (448 / amax)) (fp32 product); an all-zero block gives s_a = 0 and zero
+ * codes.  q_e4m3 [M,K] (E4M3 bit patterns), s_a fp32 [M, K/128]; K <= 24576. */
+sq_status sq_quant_fp8_per_group(const void* x_bf16, const float* inv_smooth, uint8_t* q_e4m3,
+                                 float* s_a, int64_t M, int64_t K, void* stream);
+
+/* FP8 block-scaled weights [P3b]: one scale per [128, 128] block of the
+ * folded weight f32(w[n,k]) * smooth[k] (smooth may be NULL), with the
+ * arithmetic of sq_quant_fp8_per_group over the block's 16384 values.
+ * N % 128 == 0; q_e4m3 [N,K], s_w fp32 [N/128, K/128]. */
+sq_status sq_quant_fp8_block(const void* w_bf16, const float* smooth, uint8_t* q_e4m3,
+                             float* s_w, int64_t N, int64_t K, void* stream);
+
+/* FP8 block-scaled GEMM [P3b]: tcgen05 E4M3 x E4M3 products accumulated in
+ * fp32 per 128-wide K block (P_kb; the accumulation order inside a block is
+ * the tensor core's), then acc = fmaf(P_kb, f32(s_a[m,kb] * s_w[n/128,kb]),
+ * acc) for kb ascending, y = bf16_rne(acc).  N % 128 == 0.  Workspace as for
+ * w8a8_scaled_mm (SQ_OP_FP8BLK; currently always 0). */
+sq_status fp8_block_mm(const uint8_t* q_a, const float* s_a, const uint8_t* q_w,
+                       const float* s_w, void* y_bf16, int64_t M, int64_t N, int64_t K,
+                       void* workspace, size_t ws_bytes, void* stream);
 
 /* Bytes of workspace an operation needs for these sizes (0 = none). */
 size_t sq_workspace_bytes(int op, int64_t M, int64_t N, int64_t K);

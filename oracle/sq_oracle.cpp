@@ -601,6 +601,11 @@ int oracle_fp8_block_mm(const uint8_t* q_a, const float* s_a, const uint8_t* q_w
   const int64_t G = 128;
   if (M < 0 || N < 0 || K < 0 || (N % G) || (K % G) || !rows_ok(rows, nrows, M)) return -1;
   const int64_t nkb = K / G;
+  // decoded weights (each code's exact value), decoded once
+  std::vector<double> wd(static_cast<size_t>(N * K));
+  parallel_for(N, [&](int64_t n) {
+    for (int64_t k = 0; k < K; ++k) wd[n * K + k] = e4m3_to_f32(q_w[n * K + k]);
+  });
   parallel_for(nrows, [&](int64_t r) {
     const int64_t m = row_of(rows, r);
     std::vector<double> a(static_cast<size_t>(K));
@@ -610,7 +615,7 @@ int oracle_fp8_block_mm(const uint8_t* q_a, const float* s_a, const uint8_t* q_w
       for (int64_t kb = 0; kb < nkb; ++kb) {
         double part = 0.0, pmag = 0.0;   // exact: products have 8 significant bits
         for (int64_t k = kb * G; k < (kb + 1) * G; ++k) {
-          const double p = a[k] * static_cast<double>(e4m3_to_f32(q_w[n * K + k]));
+          const double p = a[k] * wd[n * K + k];
           part += p;
           pmag += std::fabs(p);
         }

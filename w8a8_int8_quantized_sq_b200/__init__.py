@@ -14,6 +14,14 @@ Functions (CUDA tensors in, CUDA tensors out, on the current stream):
   linear_w8a8(x, inv_s, q_w, s_ch)     -> y bf16 [M,N] (quant + GEMM)
   smooth_factors(x, w, cap, floor)     -> (s f32 [K], inv_s f32 [K])
   quant_weight(w, smooth, group)       -> (q_w int8 [N,K], scales)
+  fold_norm_weight(w_norm, inv_s)      -> gamma f32 [K]
+  rmsnorm_quant(h, gamma, eps, group)  -> (q int8 [M,K], scales, inv_rms f32 [M])
+  quant_per_group(x, inv_s)            -> (q_a int8 [M,K], s_a f32 [M,K/128])
+  w8a8_pg128_mm(q_a, s_a, q_w, s_blk)  -> y bf16 [M,N]
+  w8a16_group_mm(x, q_w, s_grp)        -> y bf16 [M,N]
+  quant_fp8_per_group(x, inv_s)        -> (q e4m3 uint8 [M,K], s_a f32 [M,K/128])
+  quant_fp8_block(w, smooth)           -> (q e4m3 uint8 [N,K], s_w f32 [N/128,K/128])
+  fp8_block_mm(q_a, s_a, q_w, s_w)     -> y bf16 [M,N]
 """
 from __future__ import annotations
 
@@ -28,6 +36,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libsqint8.so")
 
 OP_W8A8, OP_GS128, OP_W8A16, OP_W8A8_I32 = 0, 1, 2, 3
+OP_PG128, OP_FP8BLK, OP_W8A16_GROUP = 4, 5, 6
 _STATUS = {0: "ok", 1: "null pointer", 2: "unsupported shape", 3: "pointer not 16-byte aligned",
            4: "workspace missing or too small", 5: "CUDA error", 6: "kernel wait timed out"}
 
@@ -67,6 +76,14 @@ def lib() -> ctypes.CDLL:
                 "sq_check_device_error": [ctypes.c_int],
                 "sq_set_overlap": [ctypes.c_int],
                 "sq_describe_plan": [ctypes.c_int, i64, i64, i64, ctypes.c_int, vp],
+                "sq_fold_norm_weight": [vp, ctypes.c_int, vp, vp, i64, vp],
+                "sq_rmsnorm_quant": [vp, vp, ctypes.c_float, i64, vp, vp, vp, i64, i64, vp],
+                "sq_quant_per_group": [vp, vp, vp, vp, i64, i64, vp],
+                "w8a8_pg128_mm": [vp, vp, vp, vp, vp, i64, i64, i64, vp, sz, vp],
+                "w8a16_group_mm": [vp, vp, vp, vp, i64, i64, i64, vp, sz, vp],
+                "sq_quant_fp8_per_group": [vp, vp, vp, vp, i64, i64, vp],
+                "sq_quant_fp8_block": [vp, vp, vp, vp, i64, i64, vp],
+                "fp8_block_mm": [vp, vp, vp, vp, vp, i64, i64, i64, vp, sz, vp],
             }
             for name, args in sig.items():
                 f = getattr(L, name)
@@ -83,7 +100,9 @@ def lib() -> ctypes.CDLL:
 EXPORTS = ("sq_quant_per_token", "w8a8_scaled_mm", "w8a8_gs128_mm", "w8a16_mm",
            "sq_workspace_bytes", "w8a8_mm_i32", "sq_smooth_factors", "sq_quant_weight",
            "sq_check_device_error", "sq_status_string", "w8a8_scaled_mm_noalloc",
-           "sq_w8a8_linear", "sq_set_overlap", "sq_describe_plan")
+           "sq_w8a8_linear", "sq_set_overlap", "sq_describe_plan", "sq_fold_norm_weight",
+           "sq_rmsnorm_quant", "sq_quant_per_group", "w8a8_pg128_mm", "w8a16_group_mm",
+           "sq_quant_fp8_per_group", "sq_quant_fp8_block", "fp8_block_mm")
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -225,6 +244,92 @@ def quant_weight(w, smooth: Optional[torch.Tensor] = None, group: int = 0):
     _check("sq_quant_weight", lib().sq_quant_weight(
         _ptr(w), _ptr(smooth), _ptr(q), _ptr(sc), N, K, group, _stream(w.device)))
     return q, sc
+
+
+def fold_norm_weight(w_norm, inv_s: Optional[torch.Tensor] = None, zero_centered: bool = True):
+    """gamma f32 [K]: the (zero-centred) norm weight with 1/s folded in."""
+    K = w_norm.numel()
+    g = torch.empty((K,), dtype=torch.float32, device=w_norm.device)
+    _check("sq_fold_norm_weight", lib().sq_fold_norm_weight(
+        _ptr(w_norm), 1 if zero_centered else 0, _ptr(inv_s), _ptr(g), K, _stream(w_norm.device)))
+    return g
+
+
+def rmsnorm_quant(h, gamma, eps: float, group: int = 0, out=None):
+    """Fused RMSNorm + fold + INT8 quantisation: (q, scales, inv_rms); group 0 =
+    one scale per token, 128 = one per 128 columns."""
+    M, K = h.shape
+    if out is None:
+        q = torch.empty((M, K), dtype=torch.int8, device=h.device)
+        sc = torch.empty((M,) if group in (0, K) else (M, K // group), dtype=torch.float32,
+                         device=h.device)
+        r = torch.empty((M,), dtype=torch.float32, device=h.device)
+    else:
+        q, sc, r = out
+    _check("sq_rmsnorm_quant", lib().sq_rmsnorm_quant(
+        _ptr(h), _ptr(gamma), eps, group, _ptr(q), _ptr(sc), _ptr(r), M, K, _stream(h.device)))
+    return q, sc, r
+
+
+def quant_per_group(x, inv_s: Optional[torch.Tensor] = None):
+    M, K = x.shape
+    q = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    s = torch.empty((M, K // 128), dtype=torch.float32, device=x.device)
+    _check("sq_quant_per_group", lib().sq_quant_per_group(
+        _ptr(x), _ptr(inv_s), _ptr(q), _ptr(s), M, K, _stream(x.device)))
+    return q, s
+
+
+def w8a8_pg128_mm(q_a, s_a, q_w, s_blk):
+    M, K = q_a.shape
+    N = q_w.shape[0]
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=q_a.device)
+    ws, wsb = workspace(OP_PG128, M, N, K, q_a.device)
+    _check("w8a8_pg128_mm", lib().w8a8_pg128_mm(
+        _ptr(q_a), _ptr(s_a), _ptr(q_w), _ptr(s_blk), _ptr(y), M, N, K, _ptr(ws), wsb,
+        _stream(q_a.device)))
+    return y
+
+
+def w8a16_group_mm(x, q_w, s_grp):
+    M, K = x.shape
+    N = q_w.shape[0]
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    ws, wsb = workspace(OP_W8A16_GROUP, M, N, K, x.device)
+    _check("w8a16_group_mm", lib().w8a16_group_mm(
+        _ptr(x), _ptr(q_w), _ptr(s_grp), _ptr(y), M, N, K, _ptr(ws), wsb, _stream(x.device)))
+    return y
+
+
+def quant_fp8_per_group(x, inv_s: Optional[torch.Tensor] = None):
+    """(q E4M3 bit patterns uint8 [M,K], s_a f32 [M, K/128])."""
+    M, K = x.shape
+    q = torch.empty((M, K), dtype=torch.uint8, device=x.device)
+    s = torch.empty((M, K // 128), dtype=torch.float32, device=x.device)
+    _check("sq_quant_fp8_per_group", lib().sq_quant_fp8_per_group(
+        _ptr(x), _ptr(inv_s), _ptr(q), _ptr(s), M, K, _stream(x.device)))
+    return q, s
+
+
+def quant_fp8_block(w, smooth: Optional[torch.Tensor] = None):
+    """(q E4M3 bit patterns uint8 [N,K], s_w f32 [N/128, K/128])."""
+    N, K = w.shape
+    q = torch.empty((N, K), dtype=torch.uint8, device=w.device)
+    s = torch.empty((N // 128, K // 128), dtype=torch.float32, device=w.device)
+    _check("sq_quant_fp8_block", lib().sq_quant_fp8_block(
+        _ptr(w), _ptr(smooth), _ptr(q), _ptr(s), N, K, _stream(w.device)))
+    return q, s
+
+
+def fp8_block_mm(q_a, s_a, q_w, s_w):
+    M, K = q_a.shape
+    N = q_w.shape[0]
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=q_a.device)
+    ws, wsb = workspace(OP_FP8BLK, M, N, K, q_a.device)
+    _check("fp8_block_mm", lib().fp8_block_mm(
+        _ptr(q_a), _ptr(s_a), _ptr(q_w), _ptr(s_w), _ptr(y), M, N, K, _ptr(ws), wsb,
+        _stream(q_a.device)))
+    return y
 
 
 class PlanInfo(ctypes.Structure):

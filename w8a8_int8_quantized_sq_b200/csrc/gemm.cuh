@@ -39,7 +39,21 @@
 
 namespace sq {
 
-enum : int { EPI_SCALE = 0, EPI_I32 = 1, EPI_GS128 = 2 };
+// Epilogues.  The three block-scaled ones MMA every 128-wide K block into a
+// fresh accumulator and promote it in registers:
+//   EPI_GS128  : acc = fmaf(f32(P), s_blk[n,kb], acc), y = bf16(acc * s_tok[m])
+//   EPI_PG128  : acc = fmaf(f32(P), f32(s_a[m,kb] * s_blk[n,kb]), acc), y = bf16(acc)
+//   EPI_FP8BLK : E4M3 operands, fp32 block partials P,
+//                acc = fmaf(P, f32(s_a[m,kb] * s_w[n/128,kb]), acc), y = bf16(acc)
+// EPI_W16G (group-wise W8A16 on the dequant-on-load path): the converter
+// warps reconstruct bf16(f32(q) * s_grp[n, k/128]) and the epilogue stores
+// the fp32 sums as they are.
+enum : int { EPI_SCALE = 0, EPI_I32 = 1, EPI_GS128 = 2, EPI_PG128 = 3, EPI_FP8BLK = 4,
+             EPI_W16G = 5 };
+
+__host__ __device__ constexpr bool is_block_scaled(int epi) {
+  return epi == EPI_GS128 || epi == EPI_PG128 || epi == EPI_FP8BLK;
+}
 
 struct GemmArgs {
   int R, C;               // MMA rows (A rows) and columns (B rows)
@@ -50,7 +64,9 @@ struct GemmArgs {
   int M, N;               // output y is [M, N] row-major
   const float* s_tok;     // [M] per-token scales (may be null: W8A16)
   const float* s_ch;      // [N] per-channel scales
-  const float* s_blk;     // [N, kb_total] block scales (EPI_GS128)
+  const float* s_blk;     // [N, kb_total] block scales (EPI_GS128, EPI_PG128);
+                          // [N/128, kb_total] (EPI_FP8BLK)
+  const float* s_a;       // [M, kb_total] per-group activation scales
   void* out;              // bf16 [M, N] or int32 [M, N]
   uint32_t* ws;           // stream-K slots [grid][2][128][BN] 32-bit words
   unsigned int* ws_cnt;   // stream-K arrival counters [num_tiles]
@@ -98,15 +114,17 @@ struct GemmCfg {
   static constexpr int RAW_BOX_BYTES = BM * 128;
   static constexpr int RAW_A_BYTES = (RK / 2) * RAW_BOX_BYTES;
   static constexpr int RAW_BYTES = RAW_A_BYTES;
-  static constexpr int NE = (EPI == EPI_GS128) ? 8 : 4;  // epilogue warps
+  static constexpr bool BLK = is_block_scaled(EPI);
+  static constexpr bool F8 = EPI == EPI_FP8BLK;          // kind::f8f6f4 (E4M3)
+  static constexpr int NE = BLK ? 8 : 4;                 // epilogue warps
   static constexpr int NCV = CONV ? 8 : 0;               // converter warps (2 per row)
   // CONV: one more warp, the producer of the B tiles (warp 2 + NE + NCV)
   static constexpr int THREADS = 64 + NE * 32 + NCV * 32 + (CONV ? 32 : 0);
-  static constexpr int NACC = (EPI == EPI_GS128) ? 4 : 2;
+  static constexpr int NACC = BLK ? 4 : 2;
   // Narrow (swapped, small-token) tiles rotate the K blocks over NSUB
   // independent accumulators, so consecutive tiny MMAs do not wait on each
   // other's result; the epilogue adds them in a fixed order.
-  static constexpr int NSUB = (SWAP && EPI != EPI_GS128) ? 4 : 1;
+  static constexpr int NSUB = (SWAP && !BLK) ? 4 : 1;
   static constexpr int ACC_COLS = NACC * NSUB * BN;
   static constexpr int A_TMEM_COLS = 32;  // one 128 x 64 bf16 A tile in tensor memory
   // CONV: an A stage holds the RK converted K blocks of one raw stage
@@ -132,12 +150,14 @@ struct GemmCfg {
   static constexpr int OFF_SBLK = (OFF_MISC + 16 + 15) / 16 * 16;
   static constexpr int PART_BYTES = BM * BN * 4;
   static constexpr int smem_bytes(int kb_total, int csplit = 0) {
-    return 1024 + OFF_SBLK + (EPI == EPI_GS128 ? kb_total * SBLK_STRIDE * 4 : 0) +
+    return 1024 + OFF_SBLK + ((EPI == EPI_GS128 || EPI == EPI_PG128) ? kb_total * SBLK_STRIDE * 4 : 0) +
            (csplit > 1 ? (csplit - 1) * PART_BYTES : 0);
   }
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N for M = 128");
-  static_assert(EPI != EPI_GS128 || (I8 && !SWAP && BN % 64 == 0), "gs128 layout");
-  static_assert(!CONV || (!I8 && SWAP && EPI == EPI_SCALE), "dequant-on-load is W8A16, swapped");
+  static_assert(!BLK || (I8 && !SWAP && BN == 128), "block-scaled layout");
+  static_assert(!CONV || (!I8 && SWAP && (EPI == EPI_SCALE || EPI == EPI_W16G)),
+                "dequant-on-load is W8A16, swapped");
+  static_assert(EPI != EPI_W16G || CONV, "group-scaled reconstruction happens on load");
   static_assert(!CONV || (RAW_BYTES % 1024 == 0 && B_BYTES % 16 == 0), "raw stage alignment");
   static_assert(!CONV || ACC_COLS + STAGES * RK * A_TMEM_COLS <= 512, "tensor memory A ring");
 
@@ -214,9 +234,13 @@ __device__ __forceinline__ void store_chunk(const GemmArgs& g, int rt, int ct, i
       for (int j = 0; j < CW; j += 8) {
         const int n = cb + j;
         if (n + 8 > g.N) break;
-        const float4 c0v = __ldg(reinterpret_cast<const float4*>(g.s_ch + n));
-        const float4 c1v = __ldg(reinterpret_cast<const float4*>(g.s_ch + n) + 1);
-        const float sc[8] = {c0v.x, c0v.y, c0v.z, c0v.w, c1v.x, c1v.y, c1v.z, c1v.w};
+        float sc[8] = {1.0f, 1.0f, 1.0f, 1.0f, 1.0f, 1.0f, 1.0f, 1.0f};  // no s_ch: unscaled
+        if (g.s_ch) {
+          const float4 c0v = __ldg(reinterpret_cast<const float4*>(g.s_ch + n));
+          const float4 c1v = __ldg(reinterpret_cast<const float4*>(g.s_ch + n) + 1);
+          sc[0] = c0v.x; sc[1] = c0v.y; sc[2] = c0v.z; sc[3] = c0v.w;
+          sc[4] = c1v.x; sc[5] = c1v.y; sc[6] = c1v.z; sc[7] = c1v.w;
+        }
         float f[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -244,7 +268,7 @@ __device__ __forceinline__ void store_chunk(const GemmArgs& g, int rt, int ct, i
       }
     } else {
       __nv_bfloat16* out = static_cast<__nv_bfloat16*>(g.out);
-      const float sc = sc_pre ? *sc_pre : __ldg(g.s_ch + n);
+      const float sc = sc_pre ? *sc_pre : (g.s_ch ? __ldg(g.s_ch + n) : 1.0f);
 #pragma unroll
       for (int j = 0; j < CW; ++j) {
         const int m = cb + j;
@@ -466,9 +490,19 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       it.init(g);
       Seg s;
       bool ok = true;
+      const int ngrp = g.kb_total / 2;  // EPI_W16G: 128-wide groups = two 64-wide K blocks
       while (ok && it.next(g, s)) {
+        const int wrow = (s.tile % g.tiles_r) * Cfg::BM + row;  // this thread's weight row
         for (int kb = s.kb0; kb < s.kb1 && ok; kb += Cfg::RK) {
           const int n = s.kb1 - kb < Cfg::RK ? s.kb1 - kb : Cfg::RK;
+          float gsc[Cfg::RK];  // EPI_W16G: the group scale of each K block of the stage
+          if constexpr (Cfg::EPI == EPI_W16G) {
+#pragma unroll
+            for (int c = 0; c < Cfg::RK; ++c)
+              gsc[c] = (wrow < g.N && c < n)
+                           ? __ldg(g.s_blk + static_cast<size_t>(wrow) * ngrp + ((kb + c) >> 1))
+                           : 0.0f;
+          }
           if (!wait_bounded(raw_full + rs, rph, abort_flag)) { ok = false; break; }
           // the A stage is free once the MMAs that read it are done
           if (!wait_bounded(empty + cs, cph ^ 1u, abort_flag)) { ok = false; break; }
@@ -486,14 +520,26 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           };
           auto convert = [&](const uint4 w0, const uint4 w1, uint32_t slot) {
             uint32_t o[16];
-            i8x4_to_bf16x4(w0.x, o[0], o[1]);
-            i8x4_to_bf16x4(w0.y, o[2], o[3]);
-            i8x4_to_bf16x4(w0.z, o[4], o[5]);
-            i8x4_to_bf16x4(w0.w, o[6], o[7]);
-            i8x4_to_bf16x4(w1.x, o[8], o[9]);
-            i8x4_to_bf16x4(w1.y, o[10], o[11]);
-            i8x4_to_bf16x4(w1.z, o[12], o[13]);
-            i8x4_to_bf16x4(w1.w, o[14], o[15]);
+            if constexpr (Cfg::EPI == EPI_W16G) {
+              const float sc = gsc[slot];
+              i8x4_scale_to_bf16x4(w0.x, sc, o[0], o[1]);
+              i8x4_scale_to_bf16x4(w0.y, sc, o[2], o[3]);
+              i8x4_scale_to_bf16x4(w0.z, sc, o[4], o[5]);
+              i8x4_scale_to_bf16x4(w0.w, sc, o[6], o[7]);
+              i8x4_scale_to_bf16x4(w1.x, sc, o[8], o[9]);
+              i8x4_scale_to_bf16x4(w1.y, sc, o[10], o[11]);
+              i8x4_scale_to_bf16x4(w1.z, sc, o[12], o[13]);
+              i8x4_scale_to_bf16x4(w1.w, sc, o[14], o[15]);
+            } else {
+              i8x4_to_bf16x4(w0.x, o[0], o[1]);
+              i8x4_to_bf16x4(w0.y, o[2], o[3]);
+              i8x4_to_bf16x4(w0.z, o[4], o[5]);
+              i8x4_to_bf16x4(w0.w, o[6], o[7]);
+              i8x4_to_bf16x4(w1.x, o[8], o[9]);
+              i8x4_to_bf16x4(w1.y, o[10], o[11]);
+              i8x4_to_bf16x4(w1.z, o[12], o[13]);
+              i8x4_to_bf16x4(w1.w, o[14], o[15]);
+            }
             tmem_st16(a_lane + (cs * Cfg::RK + slot) * Cfg::A_TMEM_COLS + half * 16, o);
           };
           if (n == Cfg::RK) {
@@ -592,7 +638,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     // The whole warp runs the loop and waits; one elected lane issues the
     // MMAs and commits.
     {
-      const uint32_t idesc = Cfg::I8 ? idesc_i8_s32(BN) : idesc_bf16_f32(BN);
+      const uint32_t idesc =
+          Cfg::F8 ? idesc_e4m3_f32(BN) : (Cfg::I8 ? idesc_i8_s32(BN) : idesc_bf16_f32(BN));
       uint32_t stage = 0, phase = 0;
       uint32_t bstage = 0, bphase = 0;  // CONV: the separate B ring
       uint32_t local = 0;
@@ -601,7 +648,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       Seg s;
       bool ok = true;
       while (ok && it.next(g, s)) {
-        if constexpr (Cfg::EPI == EPI_GS128) {
+        if constexpr (Cfg::BLK) {
           for (int kb = s.kb0; kb < s.kb1 && ok; ++kb, ++local) {
             const uint32_t p = local % NACC, u = local / NACC;
             if (!warp_wait_bounded(tempty + p, u & 1u, abort_flag)) { ok = false; break; }
@@ -612,9 +659,14 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
             const uint32_t sb = smem_u32(smB + stage * Cfg::B_BYTES);
             if (elect_one()) {
 #pragma unroll
-              for (int k = 0; k < 4; ++k)  // a fresh int32 accumulator per K block
-                mma_i8(tmem + p * BN, smem_desc_sw128(sa + k * 32), smem_desc_sw128(sb + k * 32),
-                       idesc, k > 0 ? 1u : 0u);
+              for (int k = 0; k < 4; ++k) {  // a fresh accumulator per K block
+                if constexpr (Cfg::F8)
+                  mma_f8(tmem + p * BN, smem_desc_sw128(sa + k * 32), smem_desc_sw128(sb + k * 32),
+                         idesc, k > 0 ? 1u : 0u);
+                else
+                  mma_i8(tmem + p * BN, smem_desc_sw128(sa + k * 32), smem_desc_sw128(sb + k * 32),
+                         idesc, k > 0 ? 1u : 0u);
+              }
               mma_commit(empty + stage);
               mma_commit(tfull + p);
             }
@@ -707,8 +759,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     SegIter it;
     it.init(g);
     Seg s;
-    if constexpr (Cfg::EPI == EPI_GS128) {
+    if constexpr (Cfg::BLK) {
       constexpr int CPT = Cfg::CPT;
+      constexpr bool COLSCALE = Cfg::EPI == EPI_GS128 || Cfg::EPI == EPI_PG128;
       const int h = ew / 4;
       const int col0 = h * CPT;
       const int et = ew * 32 + lane;
@@ -719,73 +772,93 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       bool ok = true;
       while (ok && it.next(g, s)) {
         const int rt = s.tile % g.tiles_r, ct = s.tile / g.tiles_r;
-        // stage this tile's block scales, transposed to [kb][n]; each thread
-        // requests a batch of its elements before storing any
-        named_bar_sync(1, nthr);
-        const int total = g.kb_total * BN;
-        for (int base = 0; base < total; base += 8 * nthr) {
-          float vals[8];
+        const int m = rt * Cfg::BM + rr;
+        if constexpr (COLSCALE) {
+          // stage this tile's block scales, transposed to [kb][n]; each thread
+          // requests a batch of its elements before storing any
+          named_bar_sync(1, nthr);
+          const int total = g.kb_total * BN;
+          for (int base = 0; base < total; base += 8 * nthr) {
+            float vals[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int idx = base + i * nthr + et;
-            const int j = idx / g.kb_total, kb = idx - j * g.kb_total;
-            const int n = ct * BN + j;
-            vals[i] = (idx < total && n < g.N)
-                          ? __ldg(g.s_blk + static_cast<size_t>(n) * g.kb_total + kb)
-                          : 0.0f;
-          }
+            for (int i = 0; i < 8; ++i) {
+              const int idx = base + i * nthr + et;
+              const int j = idx / g.kb_total, kb = idx - j * g.kb_total;
+              const int n = ct * BN + j;
+              vals[i] = (idx < total && n < g.N)
+                            ? __ldg(g.s_blk + static_cast<size_t>(n) * g.kb_total + kb)
+                            : 0.0f;
+            }
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int idx = base + i * nthr + et;
-            const int j = idx / g.kb_total, kb = idx - j * g.kb_total;
-            if (idx < total) sblk[kb * Cfg::SBLK_STRIDE + j] = vals[i];
+            for (int i = 0; i < 8; ++i) {
+              const int idx = base + i * nthr + et;
+              const int j = idx / g.kb_total, kb = idx - j * g.kb_total;
+              if (idx < total) sblk[kb * Cfg::SBLK_STRIDE + j] = vals[i];
+            }
           }
+          named_bar_sync(1, nthr);
         }
-        named_bar_sync(1, nthr);
+        // per-group activation scales of this thread's row (0 past the last row)
+        const float* sa_row =
+            (Cfg::EPI != EPI_GS128 && m < g.M) ? g.s_a + static_cast<size_t>(m) * g.kb_total : nullptr;
         float acc[CPT];
 #pragma unroll
         for (int j = 0; j < CPT; ++j) acc[j] = 0.0f;
         for (int kb = s.kb0; kb < s.kb1; ++kb, ++local) {
           const uint32_t p = local % NACC, u = local / NACC;
+          // this K block's scalar scale factors, requested before the wait
+          float sa = 0.0f, sw = 0.0f;
+          if constexpr (Cfg::EPI != EPI_GS128) sa = sa_row ? __ldg(sa_row + kb) : 0.0f;
+          if constexpr (Cfg::F8) sw = __ldg(g.s_blk + static_cast<size_t>(ct) * g.kb_total + kb);
           const bool w_ok = wait_bounded(tfull + p, u & 1u, abort_flag);
           if (named_bar_or(1, nthr, !w_ok)) { ok = false; break; }
           tc_fence_after();
-          // this K block's int32 sums (|sum| <= 128 * 127 * 127 < 2^22), then
-          // the buffer goes straight back to the MMA
+          // this K block's partial sums (int32: |sum| <= 128 * 127 * 127 <
+          // 2^22; or fp32), then the buffer goes straight back to the MMA
           static_assert(CPT == 64, "one 64-column load per K block");
           uint32_t v[64];
           tmem_ld64(lane_base + p * BN + col0, v);
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(tempty + p);
-          // exact int32 -> fp32: add the bits of 1.5 * 2^23 (the sum lands in
-          // the mantissa), subtract 1.5 * 2^23; then one rounding per step
-          const float* sk = sblk + kb * Cfg::SBLK_STRIDE + col0;
+          if constexpr (Cfg::F8) {
+            const float sc = __fmul_rn(sa, sw);
 #pragma unroll
-          for (int j = 0; j < 64; j += 4) {
-            const float4 s4 = *reinterpret_cast<const float4*>(sk + j);
-            const float sc[4] = {s4.x, s4.y, s4.z, s4.w};
+            for (int j = 0; j < 64; ++j) acc[j] = __fmaf_rn(__uint_as_float(v[j]), sc, acc[j]);
+          } else {
+            // exact int32 -> fp32: add the bits of 1.5 * 2^23 (the sum lands in
+            // the mantissa), subtract 1.5 * 2^23; then one rounding per step
+            const float* sk = sblk + kb * Cfg::SBLK_STRIDE + col0;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const float f = __fsub_rn(__uint_as_float(v[j + i] + 0x4B400000u), 12582912.0f);
-              acc[j + i] = __fmaf_rn(f, sc[i], acc[j + i]);
+            for (int j = 0; j < 64; j += 4) {
+              const float4 s4 = *reinterpret_cast<const float4*>(sk + j);
+              float sc[4] = {s4.x, s4.y, s4.z, s4.w};
+              if constexpr (Cfg::EPI == EPI_PG128) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) sc[i] = __fmul_rn(sa, sc[i]);
+              }
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const float f = __fsub_rn(__uint_as_float(v[j + i] + 0x4B400000u), 12582912.0f);
+                acc[j + i] = __fmaf_rn(f, sc[i], acc[j + i]);
+              }
             }
           }
         }
         if (!ok) break;
-        const int m = rt * Cfg::BM + rr;
         if (m < g.M) {
-          const float st = __ldg(g.s_tok + m);
+          const float st = Cfg::EPI == EPI_GS128 ? __ldg(g.s_tok + m) : 1.0f;
           __nv_bfloat16* out = static_cast<__nv_bfloat16*>(g.out) + static_cast<size_t>(m) * g.N;
 #pragma unroll
           for (int j = 0; j < CPT; j += 8) {
             const int n = ct * BN + col0 + j;
+            float o[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) o[i] = Cfg::EPI == EPI_GS128 ? __fmul_rn(acc[j + i], st) : acc[j + i];
             if (n + 8 <= g.N)
-              *reinterpret_cast<uint4*>(out + n) = make_uint4(
-                  pack_bf16x2(__fmul_rn(acc[j], st), __fmul_rn(acc[j + 1], st)),
-                  pack_bf16x2(__fmul_rn(acc[j + 2], st), __fmul_rn(acc[j + 3], st)),
-                  pack_bf16x2(__fmul_rn(acc[j + 4], st), __fmul_rn(acc[j + 5], st)),
-                  pack_bf16x2(__fmul_rn(acc[j + 6], st), __fmul_rn(acc[j + 7], st)));
+              *reinterpret_cast<uint4*>(out + n) =
+                  make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]),
+                             pack_bf16x2(o[4], o[5]), pack_bf16x2(o[6], o[7]));
           }
         }
       }
@@ -798,12 +871,13 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         const int rt = s.tile % g.tiles_r, ct = s.tile / g.tiles_r;
         // the channel scale of this thread's output row, fetched while the
         // MMAs finish (swapped layout: one weight row per thread)
-        float sc_pre = 0.0f;
+        float sc_pre = 1.0f;  // EPI_W16G: the scales were applied on load
         if constexpr (Cfg::SWAP && Cfg::EPI == EPI_SCALE) {
           const int n = rt * Cfg::BM + rr;
-          if (n < g.N) sc_pre = __ldg(g.s_ch + n);
+          if (n < g.N) sc_pre = g.s_ch ? __ldg(g.s_ch + n) : 1.0f;
         }
-        const float* scp = (Cfg::SWAP && Cfg::EPI == EPI_SCALE) ? &sc_pre : nullptr;
+        const float* scp =
+            (Cfg::SWAP && (Cfg::EPI == EPI_SCALE || Cfg::EPI == EPI_W16G)) ? &sc_pre : nullptr;
         const bool w_ok = wait_bounded(tfull + a, u & 1u, abort_flag);
         if (named_bar_or(1, nthr, !w_ok)) break;
         tc_fence_after();

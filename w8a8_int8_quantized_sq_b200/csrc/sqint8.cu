@@ -89,7 +89,15 @@ sq_status launch_status() {
 }
 
 // ---------------------------------------------------------------- planning
-enum GemmKind { GK_I8_SCALE = 0, GK_I8_I32 = 1, GK_GS128 = 2, GK_BF16 = 3, GK_W8A16_CONV = 4 };
+enum GemmKind {
+  GK_I8_SCALE = 0, GK_I8_I32 = 1, GK_GS128 = 2, GK_BF16 = 3, GK_W8A16_CONV = 4,
+  GK_PG128 = 5,        // per-group activations x gs128 weights
+  GK_FP8BLK = 6,       // E4M3 per-group activations x [128, 128] block weights
+  GK_W8A16G_CONV = 7   // group-wise W8A16, reconstructed on load (M <= 32)
+};
+
+// One 128 x 128 tile per CTA, a fresh accumulator per 128-wide K block.
+bool block_scaled(GemmKind k) { return k == GK_GS128 || k == GK_PG128 || k == GK_FP8BLK; }
 
 struct GemmPlan {
   bool pair;  // CTA-pair kernel (256 x 256 tiles per cluster of two)
@@ -123,9 +131,9 @@ bool overlap_on() { return g_overlap.load(std::memory_order_relaxed) != 0; }
 
 GemmPlan plan_gemm(GemmKind kind, int64_t M, int64_t N, int64_t K, int sms) {
   GemmPlan p{};
-  const bool i8 = kind != GK_BF16 && kind != GK_W8A16_CONV;
+  const bool i8 = kind != GK_BF16 && kind != GK_W8A16_CONV && kind != GK_W8A16G_CONV;
   p.kb_total = static_cast<int>(K / (i8 ? 128 : 64));
-  if (kind != GK_GS128 && M <= 32) {
+  if (!block_scaled(kind) && M <= 32) {
     p.swap = true;
     p.bn = M <= 16 ? 16 : 32;
     p.tiles_r = static_cast<int>((N + 127) / 128);
@@ -162,7 +170,7 @@ GemmPlan plan_gemm(GemmKind kind, int64_t M, int64_t N, int64_t K, int sms) {
     p.ws_bytes = 0;
   } else {
     p.swap = false;
-    p.bn = kind == GK_GS128 ? 128 : 256;
+    p.bn = block_scaled(kind) ? 128 : 256;
     p.tiles_r = static_cast<int>((M + 127) / 128);
     p.tiles_c = static_cast<int>((N + p.bn - 1) / p.bn);
     p.stream_k = false;
@@ -210,7 +218,7 @@ sq_status launch_gemm(const CUtensorMap& a, const CUtensorMap& b, GemmArgs g, in
   g.pdl = pdl ? 1 : 0;
   // cluster split-K needs room for the parts and every cluster resident at once;
   // otherwise the tile's parts meet in the workspace
-  if (g.csplit > 1 && (Cfg::EPI == EPI_GS128 || Cfg::CONV ||
+  if (g.csplit > 1 && (Cfg::BLK || Cfg::CONV ||
                        Cfg::smem_bytes(g.kb_total, g.csplit) > 232448))
     g.csplit = 0;
   const int smem = Cfg::smem_bytes(g.kb_total, g.csplit);
@@ -303,7 +311,8 @@ sq_status launch_gemm2(const CUtensorMap& a, const CUtensorMap& b, const GemmArg
 // act: q_a int8 [M,K] or x bf16 [M,K]; wt: q_w int8 [N,K] or bf16 [N,K].
 sq_status run_gemm(GemmKind kind, const void* act, const void* wt, const float* s_tok,
                    const float* s_ch, const float* s_blk, void* out, int64_t M, int64_t N,
-                   int64_t K, void* ws, size_t ws_bytes, cudaStream_t st, bool pdl = false) {
+                   int64_t K, void* ws, size_t ws_bytes, cudaStream_t st, bool pdl = false,
+                   const float* s_a = nullptr) {
   const int sms = num_sms();
   if (sms <= 0) return SQ_ERR_CUDA;
   const GemmPlan p = plan_gemm(kind, M, N, K, sms);
@@ -311,7 +320,7 @@ sq_status run_gemm(GemmKind kind, const void* act, const void* wt, const float* 
     return SQ_ERR_SHAPE;
   if (p.ws_bytes > 0 && (!ws || ws_bytes < p.ws_bytes)) return SQ_ERR_WORKSPACE;
   if (ws && !aligned16(ws)) return SQ_ERR_ALIGN;
-  const bool conv = kind == GK_W8A16_CONV;
+  const bool conv = kind == GK_W8A16_CONV || kind == GK_W8A16G_CONV;
   const bool bf16 = kind == GK_BF16 || conv;
   const uint32_t kbe = bf16 ? 64 : 128;
   CUtensorMap ta, tb;
@@ -345,6 +354,7 @@ sq_status run_gemm(GemmKind kind, const void* act, const void* wt, const float* 
   g.s_tok = s_tok;
   g.s_ch = s_ch;
   g.s_blk = s_blk;
+  g.s_a = s_a;
   g.out = out;
   g.ws_cnt = p.ws_bytes ? static_cast<unsigned int*>(ws) : nullptr;
   g.ws = p.ws_bytes ? reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + kCounterBytes)
@@ -372,6 +382,16 @@ sq_status run_gemm(GemmKind kind, const void* act, const void* wt, const float* 
       return launch_gemm<GemmCfg<true, 256, 4, false, EPI_I32>>(ta, tb, g, p.grid, st, pdl);
     case GK_GS128:
       return launch_gemm<GemmCfg<true, 128, 4, false, EPI_GS128>>(ta, tb, g, p.grid, st, pdl);
+    case GK_PG128:
+      return launch_gemm<GemmCfg<true, 128, 4, false, EPI_PG128>>(ta, tb, g, p.grid, st, pdl);
+    case GK_FP8BLK:
+      return launch_gemm<GemmCfg<true, 128, 4, false, EPI_FP8BLK>>(ta, tb, g, p.grid, st, pdl);
+    case GK_W8A16G_CONV:
+      if (p.bn == 16)
+        return launch_gemm<GemmCfg<false, 16, 3, true, EPI_W16G, true, 5>>(ta, tb, g, p.grid,
+                                                                          st, pdl);
+      return launch_gemm<GemmCfg<false, 32, 2, true, EPI_W16G, true, 5>>(ta, tb, g, p.grid, st,
+                                                                        pdl);
     case GK_BF16:
       // bf16 weight copies exist only for M > 32 (no swapped schedule)
       if (p.swap) return SQ_ERR_SHAPE;
@@ -391,7 +411,7 @@ sq_status run_gemm(GemmKind kind, const void* act, const void* wt, const float* 
 size_t w8a16_ws_bytes(int64_t M, int64_t N, int64_t K, int sms, size_t* w_off) {
   if (M <= 32) {
     if (w_off) *w_off = 0;
-    return plan_gemm(GK_W8A16_CONV, M, N, K, sms).ws_bytes;
+    return plan_gemm(GK_W8A16_CONV, M, N, K, sms).ws_bytes;  // same plan for GK_W8A16G_CONV
   }
   const GemmPlan p = plan_gemm(GK_BF16, M, N, K, sms);
   const size_t off = align256(p.ws_bytes > kCounterBytes ? p.ws_bytes : kCounterBytes);
@@ -411,9 +431,10 @@ sq_status launch_quant(const void* x, const float* vec, int8_t* q, float* scales
   return launch_status();
 }
 
-template <int TPR, int CH, int G>
+template <int TPR, int CH, int G, int MODE>
 sq_status launch_quant_stream(const void* x, const float* vec, int8_t* q, float* scales,
-                              int64_t rows, int64_t K, cudaStream_t st) {
+                              int64_t rows, int64_t K, cudaStream_t st, float eps,
+                              float* r_out) {
   const size_t row_bytes = static_cast<size_t>(K) * 2;
   // ring depth: about 100 KB of rows per block (two blocks per SM), at least
   // two rows per group so one is in flight while the other is processed
@@ -425,52 +446,64 @@ sq_status launch_quant_stream(const void* x, const float* vec, int8_t* q, float*
   if (sms <= 0) return SQ_ERR_CUDA;
   int64_t blocks = (rows + G - 1) / G;
   if (blocks > 2 * sms) blocks = 2 * sms;
-  auto kern = vec ? quant_stream_kernel<TPR, CH, G, true> : quant_stream_kernel<TPR, CH, G, false>;
+  auto kern = vec ? quant_stream_kernel<TPR, CH, G, true, MODE>
+                  : quant_stream_kernel<TPR, CH, G, false, MODE>;
   static std::atomic<int> smem_set[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SQ_ERR_CUDA;
   const int flag = vec ? 2 : 1;
   if ((smem_set[dev].load() & flag) == 0) {
-    if (cudaFuncSetAttribute(quant_stream_kernel<TPR, CH, G, true>,
+    if (cudaFuncSetAttribute(quant_stream_kernel<TPR, CH, G, true, MODE>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, 232448) != cudaSuccess ||
-        cudaFuncSetAttribute(quant_stream_kernel<TPR, CH, G, false>,
+        cudaFuncSetAttribute(quant_stream_kernel<TPR, CH, G, false, MODE>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, 232448) != cudaSuccess)
       return SQ_ERR_CUDA;
     smem_set[dev].fetch_or(3);
   }
   kern<<<static_cast<unsigned>(blocks), TPR * G, smem, st>>>(
-      static_cast<const __nv_bfloat16*>(x), vec, q, scales, rows, static_cast<int>(K), S);
+      static_cast<const __nv_bfloat16*>(x), vec, q, scales, rows, static_cast<int>(K), S, eps,
+      r_out);
   return launch_status();
 }
 
-template <int TPR, int G>
+template <int TPR, int G, int MODE>
 sq_status launch_quant_stream_ch(int ch, const void* x, const float* vec, int8_t* q,
-                                 float* scales, int64_t rows, int64_t K, cudaStream_t st) {
+                                 float* scales, int64_t rows, int64_t K, cudaStream_t st,
+                                 float eps, float* r_out) {
   switch (ch) {
-    case 1: return launch_quant_stream<TPR, 1, G>(x, vec, q, scales, rows, K, st);
-    case 2: return launch_quant_stream<TPR, 2, G>(x, vec, q, scales, rows, K, st);
-    case 3: return launch_quant_stream<TPR, 3, G>(x, vec, q, scales, rows, K, st);
-    case 4: return launch_quant_stream<TPR, 4, G>(x, vec, q, scales, rows, K, st);
-    case 5: return launch_quant_stream<TPR, 5, G>(x, vec, q, scales, rows, K, st);
-    default: return launch_quant_stream<TPR, 6, G>(x, vec, q, scales, rows, K, st);
+    case 1: return launch_quant_stream<TPR, 1, G, MODE>(x, vec, q, scales, rows, K, st, eps, r_out);
+    case 2: return launch_quant_stream<TPR, 2, G, MODE>(x, vec, q, scales, rows, K, st, eps, r_out);
+    case 3: return launch_quant_stream<TPR, 3, G, MODE>(x, vec, q, scales, rows, K, st, eps, r_out);
+    case 4: return launch_quant_stream<TPR, 4, G, MODE>(x, vec, q, scales, rows, K, st, eps, r_out);
+    case 5: return launch_quant_stream<TPR, 5, G, MODE>(x, vec, q, scales, rows, K, st, eps, r_out);
+    default: return launch_quant_stream<TPR, 6, G, MODE>(x, vec, q, scales, rows, K, st, eps, r_out);
   }
 }
 
-// One scale per row of K elements (K <= 24576): the streaming kernel with the
-// fewest threads per row that keeps at most 6 chunks of 16 columns (and
-// their 1/s factors) per thread.
+// Largest K the streaming kernel takes (256 threads x 6 chunks x 16 columns).
+constexpr int64_t kMaxStreamK = 256 * 16 * 6;
+
+// One row of K elements (K <= kMaxStreamK) per step: the streaming kernel with
+// the fewest threads per row that keeps at most 6 chunks of 16 columns (and
+// their 1/s factors) per thread.  MODE: QM_* bits (norm, 128-wide groups, FP8).
+template <int MODE = 0>
 sq_status quant_per_row(const void* x, const float* vec, int8_t* q, float* scales, int64_t rows,
-                        int64_t K, cudaStream_t st) {
+                        int64_t K, cudaStream_t st, float eps = 0.0f, float* r_out = nullptr) {
   const int64_t c64 = (K + 1023) / 1024, c128 = (K + 2047) / 2048, c256 = (K + 4095) / 4096;
-  if (c64 <= 6) return launch_quant_stream_ch<64, 4>(static_cast<int>(c64), x, vec, q, scales, rows, K, st);
-  if (c128 <= 6) return launch_quant_stream_ch<128, 1>(static_cast<int>(c128), x, vec, q, scales, rows, K, st);
-  return launch_quant_stream_ch<256, 1>(static_cast<int>(c256), x, vec, q, scales, rows, K, st);
+  if (c64 <= 6)
+    return launch_quant_stream_ch<64, 4, MODE>(static_cast<int>(c64), x, vec, q, scales, rows, K,
+                                               st, eps, r_out);
+  if (c128 <= 6)
+    return launch_quant_stream_ch<128, 1, MODE>(static_cast<int>(c128), x, vec, q, scales, rows,
+                                                K, st, eps, r_out);
+  return launch_quant_stream_ch<256, 1, MODE>(static_cast<int>(c256), x, vec, q, scales, rows, K,
+                                              st, eps, r_out);
 }
 
 sq_status quant_rows(const void* x, const float* vec, int8_t* q, float* scales, int64_t nseg,
                      int64_t K, int64_t group, cudaStream_t st) {
   if (nseg == 0) return SQ_OK;
-  if (group == K && K <= 256 * 16 * 6) return quant_per_row(x, vec, q, scales, nseg, K, st);
+  if (group == K && K <= kMaxStreamK) return quant_per_row(x, vec, q, scales, nseg, K, st);
   if (group == 128) {
     return vec ? launch_quant<8, true>(x, vec, q, scales, nseg, K, group, st)
                : launch_quant<8, false>(x, vec, q, scales, nseg, K, group, st);
@@ -558,6 +591,9 @@ size_t sq_workspace_bytes(int op, int64_t M, int64_t N, int64_t K) {
     case SQ_OP_W8A8_I32: return plan_gemm(GK_I8_I32, M, N, K, sms).ws_bytes;
     case SQ_OP_GS128: return plan_gemm(GK_GS128, M, N, K, sms).ws_bytes;
     case SQ_OP_W8A16: return w8a16_ws_bytes(M, N, K, sms, nullptr);
+    case SQ_OP_PG128: return plan_gemm(GK_PG128, M, N, K, sms).ws_bytes;
+    case SQ_OP_FP8BLK: return plan_gemm(GK_FP8BLK, M, N, K, sms).ws_bytes;
+    case SQ_OP_W8A16_GROUP: return w8a16_ws_bytes(M, N, K, sms, nullptr);
   }
   return 0;
 }
@@ -574,6 +610,9 @@ sq_status sq_describe_plan(int op, int64_t M, int64_t N, int64_t K, int sms,
     case SQ_OP_W8A8_I32: kind = GK_I8_I32; break;
     case SQ_OP_GS128: kind = GK_GS128; break;
     case SQ_OP_W8A16: kind = M <= 32 ? GK_W8A16_CONV : GK_BF16; break;
+    case SQ_OP_PG128: kind = GK_PG128; break;
+    case SQ_OP_FP8BLK: kind = GK_FP8BLK; break;
+    case SQ_OP_W8A16_GROUP: kind = M <= 32 ? GK_W8A16G_CONV : GK_BF16; break;
     default: return SQ_ERR_SHAPE;
   }
   const GemmPlan p = plan_gemm(kind, M, N, K, sms);
@@ -598,7 +637,9 @@ sq_status sq_describe_plan(int op, int64_t M, int64_t N, int64_t K, int sms,
     r.tile_n = 128;
     r.splits = p.splits;
   }
-  r.workspace_bytes = op == SQ_OP_W8A16 ? w8a16_ws_bytes(M, N, K, sms, nullptr) : p.ws_bytes;
+  r.workspace_bytes = (op == SQ_OP_W8A16 || op == SQ_OP_W8A16_GROUP)
+                          ? w8a16_ws_bytes(M, N, K, sms, nullptr)
+                          : p.ws_bytes;
   *out = r;
   return SQ_OK;
 }
@@ -689,6 +730,136 @@ sq_status w8a16_mm(const void* x_bf16, const int8_t* q_w, const float* s_ch, voi
   if (launch_status() != SQ_OK) return SQ_ERR_CUDA;
   // never a programmatic launch here: its weights come from the kernel just before
   return run_gemm(GK_BF16, x_bf16, wb, nullptr, s_ch, nullptr, y_bf16, M, N, K, workspace,
+                  w_off, st);
+}
+
+// ---------------------------------------------------------------------------
+// Fused RMSNorm + fold + quantisation, per-group activations, group-wise
+// W8A16 and FP8 block scaling.
+
+sq_status sq_fold_norm_weight(const void* w_norm_bf16, int zero_centered,
+                              const float* inv_smooth, float* gamma, int64_t K, void* stream) {
+  if (K <= 0 || K > kMaxK) return SQ_ERR_SHAPE;
+  if (!w_norm_bf16 || !gamma) return SQ_ERR_NULL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  fold_norm_weight_kernel<<<static_cast<unsigned>((K + 255) / 256), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(w_norm_bf16), zero_centered, inv_smooth, gamma,
+      static_cast<int>(K));
+  return launch_status();
+}
+
+sq_status sq_rmsnorm_quant(const void* h_bf16, const float* gamma, float eps, int64_t group,
+                           int8_t* q_i8, float* scales, float* inv_rms, int64_t M, int64_t K,
+                           void* stream) {
+  if (M < 0 || K <= 0 || K % 128 || K > kMaxStreamK) return SQ_ERR_SHAPE;
+  if (group != 0 && group != K && group != 128) return SQ_ERR_SHAPE;
+  if (!(eps > 0.0f) || !(eps < 3.4e38f)) return SQ_ERR_SHAPE;
+  if (M == 0) return SQ_OK;
+  if (!h_bf16 || !gamma || !q_i8 || !scales) return SQ_ERR_NULL;
+  if (!aligned16(h_bf16) || !aligned16(gamma) || !aligned16(q_i8) || !aligned16(scales))
+    return SQ_ERR_ALIGN;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (group == 128 && K != 128)
+    return quant_per_row<QM_NORM | QM_GROUP>(h_bf16, gamma, q_i8, scales, M, K, st, eps, inv_rms);
+  return quant_per_row<QM_NORM>(h_bf16, gamma, q_i8, scales, M, K, st, eps, inv_rms);
+}
+
+sq_status sq_quant_per_group(const void* x_bf16, const float* inv_smooth, int8_t* q_i8,
+                             float* s_a, int64_t M, int64_t K, void* stream) {
+  if (M < 0 || K <= 0 || K % 128 || K > kMaxK) return SQ_ERR_SHAPE;
+  if (M == 0) return SQ_OK;
+  if (!x_bf16 || !q_i8 || !s_a) return SQ_ERR_NULL;
+  if (!aligned16(x_bf16) || !aligned16(q_i8) || !aligned16(s_a) ||
+      (inv_smooth && !aligned16(inv_smooth)))
+    return SQ_ERR_ALIGN;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (K <= kMaxStreamK)
+    return quant_per_row<QM_GROUP>(x_bf16, inv_smooth, q_i8, s_a, M, K, st);
+  return quant_rows(x_bf16, inv_smooth, q_i8, s_a, M * (K / 128), K, 128, st);
+}
+
+sq_status sq_quant_fp8_per_group(const void* x_bf16, const float* inv_smooth, uint8_t* q_e4m3,
+                                 float* s_a, int64_t M, int64_t K, void* stream) {
+  if (M < 0 || K <= 0 || K % 128 || K > kMaxStreamK) return SQ_ERR_SHAPE;
+  if (M == 0) return SQ_OK;
+  if (!x_bf16 || !q_e4m3 || !s_a) return SQ_ERR_NULL;
+  if (!aligned16(x_bf16) || !aligned16(q_e4m3) || !aligned16(s_a) ||
+      (inv_smooth && !aligned16(inv_smooth)))
+    return SQ_ERR_ALIGN;
+  return quant_per_row<QM_GROUP | QM_FP8>(x_bf16, inv_smooth, reinterpret_cast<int8_t*>(q_e4m3),
+                                          s_a, M, K, static_cast<cudaStream_t>(stream));
+}
+
+sq_status sq_quant_fp8_block(const void* w_bf16, const float* smooth, uint8_t* q_e4m3,
+                             float* s_w, int64_t N, int64_t K, void* stream) {
+  if (N < 0 || K <= 0 || K % 128 || N % 128 || K > kMaxK) return SQ_ERR_SHAPE;
+  if (N == 0) return SQ_OK;
+  if (!w_bf16 || !q_e4m3 || !s_w) return SQ_ERR_NULL;
+  if (!aligned16(w_bf16) || !aligned16(q_e4m3) || !aligned16(s_w) || (smooth && !aligned16(smooth)))
+    return SQ_ERR_ALIGN;
+  if (N / 128 > 65535) return SQ_ERR_SHAPE;
+  dim3 grid(static_cast<unsigned>(K / 128), static_cast<unsigned>(N / 128));
+  fp8_block_quant_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16*>(w_bf16), smooth, q_e4m3, s_w, static_cast<int>(K));
+  return launch_status();
+}
+
+sq_status w8a8_pg128_mm(const int8_t* q_a, const float* s_a, const int8_t* q_w,
+                        const float* s_blk, void* y_bf16, int64_t M, int64_t N, int64_t K,
+                        void* workspace, size_t ws_bytes, void* stream) {
+  sq_status s = check_mnk(M, N, K);
+  if (s != SQ_OK) return s;
+  if (M == 0) return SQ_OK;
+  if (!q_a || !s_a || !q_w || !s_blk || !y_bf16) return SQ_ERR_NULL;
+  if (!aligned16(q_a) || !aligned16(s_a) || !aligned16(q_w) || !aligned16(s_blk) ||
+      !aligned16(y_bf16))
+    return SQ_ERR_ALIGN;
+  return run_gemm(GK_PG128, q_a, q_w, nullptr, nullptr, s_blk, y_bf16, M, N, K, workspace,
+                  ws_bytes, static_cast<cudaStream_t>(stream), overlap_on(), s_a);
+}
+
+sq_status fp8_block_mm(const uint8_t* q_a, const float* s_a, const uint8_t* q_w,
+                       const float* s_w, void* y_bf16, int64_t M, int64_t N, int64_t K,
+                       void* workspace, size_t ws_bytes, void* stream) {
+  sq_status s = check_mnk(M, N, K);
+  if (s != SQ_OK) return s;
+  if (N % 128) return SQ_ERR_SHAPE;
+  if (M == 0) return SQ_OK;
+  if (!q_a || !s_a || !q_w || !s_w || !y_bf16) return SQ_ERR_NULL;
+  if (!aligned16(q_a) || !aligned16(s_a) || !aligned16(q_w) || !aligned16(s_w) ||
+      !aligned16(y_bf16))
+    return SQ_ERR_ALIGN;
+  return run_gemm(GK_FP8BLK, q_a, q_w, nullptr, nullptr, s_w, y_bf16, M, N, K, workspace,
+                  ws_bytes, static_cast<cudaStream_t>(stream), overlap_on(), s_a);
+}
+
+sq_status w8a16_group_mm(const void* x_bf16, const int8_t* q_w, const float* s_grp,
+                         void* y_bf16, int64_t M, int64_t N, int64_t K, void* workspace,
+                         size_t ws_bytes, void* stream) {
+  sq_status s = check_mnk(M, N, K);
+  if (s != SQ_OK) return s;
+  if (M == 0) return SQ_OK;
+  if (!x_bf16 || !q_w || !s_grp || !y_bf16) return SQ_ERR_NULL;
+  if (!aligned16(x_bf16) || !aligned16(q_w) || !aligned16(s_grp) || !aligned16(y_bf16))
+    return SQ_ERR_ALIGN;
+  const int sms = num_sms();
+  if (sms <= 0) return SQ_ERR_CUDA;
+  size_t w_off = 0;
+  const size_t need = w8a16_ws_bytes(M, N, K, sms, &w_off);
+  if (!workspace || ws_bytes < need) return SQ_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return SQ_ERR_ALIGN;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (M <= 32)  // weight-read bound: group-scaled reconstruction on load, in the GEMM
+    return run_gemm(GK_W8A16G_CONV, x_bf16, q_w, nullptr, nullptr, s_grp, y_bf16, M, N, K,
+                    workspace, ws_bytes, st, overlap_on());
+  __nv_bfloat16* wb = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(workspace) + w_off);
+  const int64_t n16 = N * K / 16;
+  const int64_t blocks = (n16 + 255) / 256 < 4 * sms ? (n16 + 255) / 256 : 4 * sms;
+  i8_to_bf16_group_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(q_w, s_grp, wb, n16,
+                                                                         static_cast<int>(K));
+  if (launch_status() != SQ_OK) return SQ_ERR_CUDA;
+  // the reconstructed weights carry the scales: the epilogue stores the sums as they are
+  return run_gemm(GK_BF16, x_bf16, wb, nullptr, nullptr, nullptr, y_bf16, M, N, K, workspace,
                   w_off, st);
 }
 
