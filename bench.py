@@ -116,9 +116,14 @@ class ClockSampler(threading.Thread):
         if not self.ok or not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
         busy = [s for s in self.samples if s > 0]
+        bins = {}
+        for v in busy:
+            b = int(v // 100 * 100)
+            bins[b] = bins.get(b, 0) + 1
         return {"sm_mhz": statistics.median(busy or self.samples), "sm_max_mhz": self.max_mhz,
                 "reasons": [n for b, n in self.REASONS.items() if self.reasons & b and b != 0x1],
-                "samples": len(self.samples)}
+                "samples": len(self.samples),
+                "mhz_bins": {str(k): bins[k] for k in sorted(bins)}}
 
 
 # -------------------------------------------------------------------- helpers
@@ -278,7 +283,8 @@ def main():
     ap.add_argument("--no-variants", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    ap.add_argument("--profile", choices=["w8a8", "gs128", "w8a16"], default=None,
+    ap.add_argument("--profile", choices=["w8a8", "gs128", "w8a16", "pg128", "fp8", "w8a16g",
+                                          "rmsnorm"], default=None,
                     help="run one operation at --M/--N/--K for --steps calls (for ncu)")
     ap.add_argument("--M", type=int, default=4096)
     ap.add_argument("--N", type=int, default=34816)
@@ -337,6 +343,25 @@ def main():
     clocks = sampler.result()
     total_s = max_over_ranks(start.elapsed_time(end) * 1e-3)
 
+    # Sustained: the same step back to back for at least two seconds (the
+    # short loop above is a burst that ends before the power cap settles).
+    sus_steps = max(args.steps, int(2.0 / max(total_s / args.steps, 1e-6)) + 1)
+    sampler = ClockSampler(local)
+    barrier()
+    sampler.start()
+    start.record()
+    for _ in range(sus_steps):
+        step()
+    end.record()
+    barrier()
+    sus_clocks = sampler.result()
+    sus_s = max_over_ranks(start.elapsed_time(end) * 1e-3)
+    sus_tops = whole_job_tops(2.0 * M * N * K, sus_steps, world, sus_s)
+    sustained = {"value": sus_tops, "unit": "TOPS", "steps": sus_steps, "seconds": sus_s,
+                 "ms_per_step": sus_s / sus_steps * 1e3, "clocks": sus_clocks,
+                 "tops_per_ghz": (sus_tops / (sus_clocks["sm_mhz"] / 1000.0)
+                                  if sus_clocks.get("sm_mhz") else None)}
+
     # The kernels on their own, live, same inputs: CUDA events around every
     # launch on the launching stream (the GEMM timing is the roofline's).
     n_kernel = max(10, min(args.steps, 100))
@@ -361,7 +386,15 @@ def main():
     del xs
     ops_step = 2.0 * M * N * K
     value = whole_job_tops(ops_step, args.steps, world, total_s)
-    int8_peak = peaks["bf16_tflops"] * INT8_PER_BF16
+    # the dense INT8 (and FP8) tensor rate of this device, measured with the
+    # library's tcgen05 issue-rate probe; 2 x the measured BF16 matmul is kept
+    # beside it for reference
+    int8_probe = sq.mma_peak(sq.PEAK_I8)
+    fp8_probe = sq.mma_peak(sq.PEAK_F8)
+    int8_proxy = peaks["bf16_tflops"] * INT8_PER_BF16
+    int8_peak = int8_probe if int8_probe > 0 else int8_proxy
+    peaks["int8_tops"] = int8_peak
+    peaks["fp8_tops"] = fp8_probe if fp8_probe > 0 else int8_peak
     gemm_tops = ops_step / gemm_s / 1e12
 
     # ---------------- end to end through the public API, host buffers
@@ -400,10 +433,17 @@ def main():
                    "l2": "inputs larger than L2 (q_w 178 MB, x 84 MB, y 570 MB)",
                    "step": "sq_w8a8_linear (per-token quant + W8A8 GEMM, PDL)"},
         "pct_of_int8_nominal": 100.0 * value / world / INT8_NOMINAL_TOPS,
+        "burst": {"value": value, "unit": "TOPS", "steps": args.steps,
+                  "tops_per_ghz": (value / (clocks["sm_mhz"] / 1000.0)
+                                   if clocks.get("sm_mhz") else None)},
+        "sustained": sustained,
         "roofline": {"bound": "tensor", "kernel": "gemm2_kernel (W8A8, CTA pairs, 256x256 tiles)",
                      "achieved": gemm_tops, "peak": int8_peak, "unit": "TOPS",
                      "frac": gemm_tops / int8_peak,
-                     "peak_source": f"{peaks['source']} bf16 burst x {INT8_PER_BF16:g}",
+                     "peak_source": "measured: tcgen05.mma kind::i8 issue-rate probe (sq_mma_peak, "
+                                    "all SMs, burst)",
+                     "peak_bf16x2": int8_proxy,
+                     "frac_of_bf16x2": gemm_tops / int8_proxy,
                      "frac_of_sustained": gemm_tops / (peaks["bf16_tflops_sustained"] * INT8_PER_BF16),
                      "traffic": gemm_traffic(),
                      "algorithmic_bytes": algo_bytes_w8a8(M, N, K)},
@@ -413,14 +453,16 @@ def main():
                       "peak_gbs": peaks["hbm_gbs"],
                       "frac": algo_bytes_quant(M, K) / quant_s / 1e9 / peaks["hbm_gbs"]},
         "e2e": e2e,
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": 2 * args.steps,  # per timed step: the quant kernel and the GEMM
         "clocks": clocks,
     }
     del x, q_w, y
     torch.cuda.empty_cache()
 
+    line["measured_peaks"] = {"int8_tops": int8_probe, "fp8_tops": fp8_probe,
+                              "hbm_gbs": peaks["hbm_gbs"], "bf16_tflops": peaks["bf16_tflops"]}
     if not args.no_variants:
-        line["variants"] = variants(sq, inputs, dev, peaks)
+        line["variants"] = variants(sq, inputs, dev, peaks) + variants_next(sq, inputs, dev, peaks)
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rows, nt, run = oracle_sample(wl, target_s=args.cpu_seconds)
@@ -460,6 +502,25 @@ def profile_case(args):
         q_a, s_tok = sq.quant_per_token(x, None)
         q_ws = [q_w] + [q_w.clone() for _ in range(copies - 1)]
         fn = lambda i: sq.w8a8_gs128_mm(q_a, s_tok, q_ws[i % copies], s_blk)  # noqa: E731
+    elif args.profile == "pg128":
+        q_w, s_blk = sq.quant_weight(w, None, group=128)
+        q_a, s_a = sq.quant_per_group(x, None)
+        q_ws = [q_w] + [q_w.clone() for _ in range(copies - 1)]
+        fn = lambda i: sq.w8a8_pg128_mm(q_a, s_a, q_ws[i % copies], s_blk)  # noqa: E731
+    elif args.profile == "fp8":
+        q_w, s_w = sq.quant_fp8_block(w)
+        q_a, s_a = sq.quant_fp8_per_group(x, None)
+        q_ws = [q_w] + [q_w.clone() for _ in range(copies - 1)]
+        fn = lambda i: sq.fp8_block_mm(q_a, s_a, q_ws[i % copies], s_w)  # noqa: E731
+    elif args.profile == "w8a16g":
+        q_w, s_grp = sq.quant_weight(w, None, group=128)
+        q_ws = [q_w] + [q_w.clone() for _ in range(copies - 1)]
+        fn = lambda i: sq.w8a16_group_mm(x, q_ws[i % copies], s_grp)  # noqa: E731
+    elif args.profile == "rmsnorm":
+        s, inv = sq.smooth_factors(x, w)
+        gamma = sq.fold_norm_weight(w[0].contiguous(), inv)
+        xs = [x] + [x.clone() for _ in range(2)]
+        fn = lambda i: sq.rmsnorm_quant(xs[i % 3], gamma, 1e-6)  # noqa: E731
     else:
         q_w, s_ch = sq.quant_weight(w, None)
         q_ws = [q_w] + [q_w.clone() for _ in range(copies - 1)]
@@ -529,7 +590,7 @@ def variants(sq, inputs, dev, peaks):
                                               s_blk), 2 * copies)
     tq = time_graph(lambda i: sq.quant_per_token(x, None), 2 * copies)
     ops = 2.0 * wl.M * wl.N * wl.K
-    int8_peak = peaks["bf16_tflops"] * INT8_PER_BF16
+    int8_peak = peaks.get("int8_tops", peaks["bf16_tflops"] * INT8_PER_BF16)
     out.append({"workload": wl.name, "metric": "TOPS (gs128 GEMM)", "value": ops / t / 1e12,
                 "unit": "TOPS", "us_per_call": t * 1e6, "frac_of_int8_peak": ops / t / 1e12 / int8_peak,
                 "tops_incl_quant": ops / (t + tq) / 1e12, "quant_us": tq * 1e6,
@@ -565,6 +626,99 @@ def variants(sq, inputs, dev, peaks):
             fl = 2.0 * M * wl.N * wl.K
             out.append({"workload": f"{wl.name}_M{M}", "metric": "TFLOP/s (bf16 tensor)",
                         "value": fl / t / 1e12, "unit": "TFLOP/s", "us_per_call": t * 1e6,
+                        "frac_of_bf16_peak": fl / t / 1e12 / peaks["bf16_tflops"],
+                        "tokens_per_s": M / t})
+        del x
+    del qws, q_w
+    torch.cuda.empty_cache()
+    return out
+
+
+def variants_next(sq, inputs, dev, peaks):
+    """The next rows: fused RMSNorm + fold + quantisation, per-group INT8 and
+    FP8 activation quantisation, per-group x gs128 and FP8 block GEMMs, and
+    group-wise W8A16; each timed alone, inputs rotating over more than L2."""
+    out = []
+    hbm = peaks["hbm_gbs"]
+    l2 = 126 * 2 ** 20
+
+    # prefill hidden state, M=8192 K=5120: the norm / quantisation kernels
+    wl = inputs.workload(2)
+    M, K = wl.M, wl.K
+    x = wl.make_x().to(dev)
+    w = wl.make_w().to(dev)
+    _, inv = sq.smooth_factors(x, w)
+    del w
+    w_norm = inputs.gen_w(1, K, inputs.SEED_BASE + 77, sigma=0.1)[0].contiguous().to(dev)
+    gamma = sq.fold_norm_weight(w_norm, inv)
+    xs = [x, x.clone(), x.clone()]
+    for group in (0, 128):
+        t = time_graph(lambda i: sq.rmsnorm_quant(xs[i % 3], gamma, 1e-6, group), 12, reps=3)
+        nsc = M if group == 0 else M * (K // 128)
+        byt = 2 * M * K + 4 * K + M * K + 4 * nsc + 4 * M
+        out.append({"workload": f"rmsnorm_quant_M{M}_K{K}_" + ("per_token" if group == 0 else "g128"),
+                    "metric": "GB/s (algorithmic bytes)", "value": byt / t / 1e9, "unit": "GB/s",
+                    "us_per_call": t * 1e6, "frac_of_hbm": byt / t / 1e9 / hbm,
+                    "tokens_per_s": M / t,
+                    "timing": "CUDA graph of 12 back-to-back launches over 3 input copies"})
+    for name, fn in (("quant_per_group_int8", lambda i: sq.quant_per_group(xs[i % 3], inv)),
+                     ("quant_per_group_fp8", lambda i: sq.quant_fp8_per_group(xs[i % 3], inv))):
+        t = time_graph(fn, 12, reps=3)
+        byt = 2 * M * K + 4 * K + M * K + 4 * M * (K // 128)
+        out.append({"workload": f"{name}_M{M}_K{K}", "metric": "GB/s (algorithmic bytes)",
+                    "value": byt / t / 1e9, "unit": "GB/s", "us_per_call": t * 1e6,
+                    "frac_of_hbm": byt / t / 1e9 / hbm, "tokens_per_s": M / t})
+    del xs, x, gamma
+
+    # block-scaled GEMMs at the gs128 workload's shape (M=2048, K=5120, N=5120)
+    wl = inputs.workload(3)
+    M, N, K = wl.M, wl.N, wl.K
+    x = wl.make_x().to(dev)
+    w = wl.make_w().to(dev)
+    q_w, s_blk = sq.quant_weight(w, None, group=128)
+    qf_w, s_w = sq.quant_fp8_block(w)
+    del w
+    q_a, s_a = sq.quant_per_group(x, None)
+    qf_a, sf_a = sq.quant_fp8_per_group(x, None)
+    copies = max(2, -(-3 * l2 // (q_w.numel() + q_a.numel())))
+    ops = 2.0 * M * N * K
+    sets = [(q_a.clone(), q_w.clone()) for _ in range(copies)]
+    t = time_graph(lambda i: sq.w8a8_pg128_mm(sets[i % copies][0], s_a, sets[i % copies][1], s_blk),
+                   2 * copies)
+    out.append({"workload": f"pg128_w8a8_M{M}_K{K}_N{N}", "metric": "TOPS (per-group x gs128 GEMM)",
+                "value": ops / t / 1e12, "unit": "TOPS", "us_per_call": t * 1e6,
+                "frac_of_int8_peak": ops / t / 1e12 / peaks["int8_tops"], "weight_copies": copies})
+    del sets
+    sets = [(qf_a.clone(), qf_w.clone()) for _ in range(copies)]
+    t = time_graph(lambda i: sq.fp8_block_mm(sets[i % copies][0], sf_a, sets[i % copies][1], s_w),
+                   2 * copies)
+    out.append({"workload": f"fp8_block_M{M}_K{K}_N{N}", "metric": "TOPS (FP8 block GEMM)",
+                "value": ops / t / 1e12, "unit": "TOPS", "us_per_call": t * 1e6,
+                "frac_of_fp8_peak": ops / t / 1e12 / peaks["fp8_tops"], "weight_copies": copies})
+    del sets, q_w, qf_w, q_a, qf_a, x
+
+    # group-wise W8A16 down_proj (K=17408, N=5120), M = 1, 16, 8192
+    wl = inputs.workload(4)
+    w = wl.make_w().to(dev)
+    q_w, s_grp = sq.quant_weight(w, None, group=128)
+    del w
+    copies = max(2, -(-3 * l2 // q_w.numel()))
+    qws = [q_w] + [q_w.clone() for _ in range(copies - 1)]
+    for M in inputs.W8A16_M_VALUES:
+        x = wl.make_x(M).to(dev)
+        if M <= 16:
+            t = time_graph(lambda i: sq.w8a16_group_mm(x, qws[i % copies], s_grp), 4 * copies)
+            byt = 2 * M * wl.K + wl.N * wl.K + 4 * wl.N * (wl.K // 128) + 2 * M * wl.N
+            out.append({"workload": f"w8a16_group_K{wl.K}_N{wl.N}_M{M}",
+                        "metric": "GB/s (algorithmic bytes)", "value": byt / t / 1e9,
+                        "unit": "GB/s", "us_per_call": t * 1e6, "frac_of_hbm": byt / t / 1e9 / hbm,
+                        "tokens_per_s": M / t, "weight_copies": copies})
+        else:
+            t = time_batches(lambda i: sq.w8a16_group_mm(x, qws[i % 2], s_grp), 10)
+            fl = 2.0 * M * wl.N * wl.K
+            out.append({"workload": f"w8a16_group_K{wl.K}_N{wl.N}_M{M}",
+                        "metric": "TFLOP/s (bf16 tensor)", "value": fl / t / 1e12,
+                        "unit": "TFLOP/s", "us_per_call": t * 1e6,
                         "frac_of_bf16_peak": fl / t / 1e12 / peaks["bf16_tflops"],
                         "tokens_per_s": M / t})
         del x

@@ -240,8 +240,10 @@ sq_status sq_quant_weight(const void* w_bf16, const float* smooth, int8_t* q_w, 
 
 /* Overlap of consecutive kernels (programmatic dependent launch; the pages
  * have no counterpart: it is a launch policy of this library).  enable != 0:
- * from now on, in this process, w8a8_scaled_mm, w8a8_mm_i32, w8a8_gs128_mm
- * and w8a16_mm (M <= 32) launch their GEMM so that it may start while the
+ * from now on, for calls made from the calling host thread only (other
+ * threads keep the default), w8a8_scaled_mm, w8a8_mm_i32, w8a8_gs128_mm,
+ * w8a8_pg128_mm, fp8_block_mm, w8a16_mm and w8a16_group_mm (M <= 32) launch
+ * their GEMM so that it may start while the
  * kernel before it on the stream is still running: it requests its WEIGHT
  * tiles (q_w) at once and reads everything else (activations, scales,
  * workspace, output) only after that kernel has completed.  Enable it only
@@ -258,7 +260,9 @@ sq_status sq_set_overlap(int enable);
  * 2 = swapped small-M tiles on stream-K ranges (partial tiles meet in the
  * workspace), 3 = swapped small-M tiles whose K parts meet inside a
  * thread-block cluster (a call falls back to 2 when the device cannot hold
- * every cluster at once or the parts do not fit in shared memory).
+ * every cluster at once or the parts do not fit in shared memory),
+ * 4 = block-scaled CTA pairs (gs128: 128 tokens x 256 channels, FP8 blocks:
+ * 256 tokens x 128 channels per pair tile).
  * tile_m x tile_n: tokens x output channels per tile.  grid: CTAs (for
  * kernel 0 an upper bound: the launch takes the active-cluster limit).
  * splits: K parts per tile when every CTA owns one part of one tile, 0 when
@@ -276,6 +280,26 @@ typedef struct {
 
 sq_status sq_describe_plan(int op, int64_t M, int64_t N, int64_t K, int sms,
                            sq_plan_info* out);
+
+/* Tensor-pipe issue-rate probe (the pages have no counterpart: it measures
+ * the roofline denominator of this device).  Launches, asynchronously on
+ * `stream`, one CTA pair per two SMs (all resident at once), each issuing
+ * `iters` back-to-back tcgen05.mma cta_group::2 instructions (M = 256,
+ * N = 256, 32 bytes of K) from shared memory: kind 0 = INT8 (kind::i8,
+ * int32 accumulators), 1 = FP8 E4M3 (kind::f8f6f4, fp32), 2 = BF16
+ * (kind::f16, fp32).  *ops_per_launch receives the launch's multiply-add
+ * count x 2; time the launch with events on `stream` and divide.
+ * 2 <= iters <= 2^24. */
+sq_status sq_mma_peak(int kind, int iters, void* stream, double* ops_per_launch);
+
+/* Self-test of the timeout path (the pages have no counterpart).  Launches on
+ * `stream` one thread that waits, with a limit of limit_cycles SM clock
+ * cycles (0 < limit_cycles <= 4e9), on a barrier that nothing arrives on.
+ * The wait gives up exactly as a GEMM role's wait does: it raises the kernel's
+ * abort flag and latches the device error word, so sq_check_device_error
+ * then returns SQ_ERR_TIMEOUT.  gave_up (device int) receives 1 when the
+ * wait gave up through its own limit.  Nothing else runs in that kernel. */
+sq_status sq_selftest_wait_timeout(int64_t limit_cycles, int* gave_up, void* stream);
 
 /* Diagnostics ------------------------------------------------------------ */
 

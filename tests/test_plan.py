@@ -56,10 +56,21 @@ def test_long_k_small_m_uses_stream_k():
     assert plan(W8A8, 8, 5120, 17408)["kernel"] == 2
 
 
-def test_gs128_and_large_m_w8a16():
+def test_block_scaled_pairs_and_large_m_w8a16():
+    # gs128 on CTA pairs, weights as the MMA's A operand: 128 tokens x 256
+    # channels per pair tile, 16 x 20 = 320 tiles over 74 pairs
     p = plan(GS128, 2048, 5120, 5120)
     assert (p["kernel"], p["tile_m"], p["tile_n"], p["grid"], p["workspace_bytes"]) == \
-        (1, 128, 128, B200_SMS, 0)
+        (4, 128, 256, B200_SMS, 0)
+    # FP8 blocks: tokens as A, 256 tokens x 128 channels (one weight block)
+    p = plan(sq.OP_FP8BLK, 2048, 5120, 5120)
+    assert (p["kernel"], p["tile_m"], p["tile_n"]) == (4, 256, 128)
+    # per-group activations x gs128 weights: one CTA per 128 x 128 tile
+    p = plan(sq.OP_PG128, 2048, 5120, 5120)
+    assert (p["kernel"], p["tile_m"], p["tile_n"], p["grid"]) == (1, 128, 128, B200_SMS)
+    # group-wise W8A16 plans like per-channel W8A16
+    for M in (1, 16, 8192):
+        assert plan(sq.OP_W8A16_GROUP, M, 5120, 17408) == plan(W8A16, M, 5120, 17408)
     # M > 32: the weights are converted into a bf16 copy in the workspace
     p = plan(W8A16, 8192, 5120, 17408)
     assert p["kernel"] == 0 and p["workspace_bytes"] >= 5120 * 17408 * 2

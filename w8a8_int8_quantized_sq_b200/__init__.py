@@ -84,6 +84,8 @@ def lib() -> ctypes.CDLL:
                 "sq_quant_fp8_per_group": [vp, vp, vp, vp, i64, i64, vp],
                 "sq_quant_fp8_block": [vp, vp, vp, vp, i64, i64, vp],
                 "fp8_block_mm": [vp, vp, vp, vp, vp, i64, i64, i64, vp, sz, vp],
+                "sq_mma_peak": [ctypes.c_int, ctypes.c_int, vp, vp],
+                "sq_selftest_wait_timeout": [i64, vp, vp],
             }
             for name, args in sig.items():
                 f = getattr(L, name)
@@ -102,7 +104,8 @@ EXPORTS = ("sq_quant_per_token", "w8a8_scaled_mm", "w8a8_gs128_mm", "w8a16_mm",
            "sq_check_device_error", "sq_status_string", "w8a8_scaled_mm_noalloc",
            "sq_w8a8_linear", "sq_set_overlap", "sq_describe_plan", "sq_fold_norm_weight",
            "sq_rmsnorm_quant", "sq_quant_per_group", "w8a8_pg128_mm", "w8a16_group_mm",
-           "sq_quant_fp8_per_group", "sq_quant_fp8_block", "fp8_block_mm")
+           "sq_quant_fp8_per_group", "sq_quant_fp8_block", "fp8_block_mm", "sq_mma_peak",
+           "sq_selftest_wait_timeout")
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -349,11 +352,43 @@ def describe_plan(op: int, M: int, N: int, K: int, sms: int) -> dict:
 
 
 def set_overlap(enable: bool) -> None:
-    """Process-wide launch policy (sq_set_overlap): when on, the GEMM entry
-    points may start streaming their weights while the preceding kernel on the
-    stream still runs.  Only for callers whose preceding kernel never writes
-    the weights of the next call."""
+    """Launch policy of the calling host thread (sq_set_overlap): when on, the
+    GEMM entry points may start streaming their weights while the preceding
+    kernel on the stream still runs.  Only for callers whose preceding kernel
+    never writes the weights of the next call."""
     _check("sq_set_overlap", lib().sq_set_overlap(1 if enable else 0))
+
+
+PEAK_I8, PEAK_F8, PEAK_BF16 = 0, 1, 2
+
+
+def mma_peak(kind: int = PEAK_I8, iters: int = 8192, device=None) -> float:
+    """Measured dense tensor throughput (tera-ops/s) of the current device
+    for one MMA kind: sq_mma_peak launched on the current stream and timed
+    with CUDA events on that stream (best of three launches after a warm-up)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    ops = ctypes.c_double(0.0)
+    best = 0.0
+    for i in range(4):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        _check("sq_mma_peak", lib().sq_mma_peak(kind, iters, _stream(dev), ctypes.byref(ops)))
+        b.record()
+        b.synchronize()
+        if i > 0:
+            best = max(best, ops.value / (a.elapsed_time(b) * 1e-3) / 1e12)
+    return best
+
+
+def selftest_wait_timeout(limit_cycles: int = 2_000_000, device=None) -> int:
+    """Run the timeout self-test kernel (sq_selftest_wait_timeout) and return
+    its gave_up flag (1: the wait gave up through its own limit).  The device
+    error word is left set: check_device_error() then raises SQ_ERR_TIMEOUT."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    flag = torch.full((1,), -1, dtype=torch.int32, device=dev)
+    _check("sq_selftest_wait_timeout",
+           lib().sq_selftest_wait_timeout(limit_cycles, _ptr(flag), _stream(dev)))
+    return int(flag.item())
 
 
 def check_device_error(reset: bool = True) -> None:

@@ -804,12 +804,19 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         float acc[CPT];
 #pragma unroll
         for (int j = 0; j < CPT; ++j) acc[j] = 0.0f;
+        // this thread's scalar scale factors of a K block (per-group
+        // activations; FP8: times the tile's weight-block scale)
+        auto row_scale = [&](int kb) -> float {
+          float sa = 0.0f;
+          if constexpr (Cfg::EPI != EPI_GS128) sa = sa_row ? __ldg(sa_row + kb) : 0.0f;
+          if constexpr (Cfg::F8)
+            sa = __fmul_rn(sa, __ldg(g.s_blk + static_cast<size_t>(ct) * g.kb_total + kb));
+          return sa;
+        };
+        float sa_next = row_scale(s.kb0);
         for (int kb = s.kb0; kb < s.kb1; ++kb, ++local) {
           const uint32_t p = local % NACC, u = local / NACC;
-          // this K block's scalar scale factors, requested before the wait
-          float sa = 0.0f, sw = 0.0f;
-          if constexpr (Cfg::EPI != EPI_GS128) sa = sa_row ? __ldg(sa_row + kb) : 0.0f;
-          if constexpr (Cfg::F8) sw = __ldg(g.s_blk + static_cast<size_t>(ct) * g.kb_total + kb);
+          const float sa = sa_next;
           const bool w_ok = wait_bounded(tfull + p, u & 1u, abort_flag);
           if (named_bar_or(1, nthr, !w_ok)) { ok = false; break; }
           tc_fence_after();
@@ -821,8 +828,11 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(tempty + p);
+          // the next K block's scales, requested after the release (a
+          // releasing arrive would otherwise wait for the load)
+          if (kb + 1 < s.kb1) sa_next = row_scale(kb + 1);
           if constexpr (Cfg::F8) {
-            const float sc = __fmul_rn(sa, sw);
+            const float sc = sa;
 #pragma unroll
             for (int j = 0; j < 64; ++j) acc[j] = __fmaf_rn(__uint_as_float(v[j]), sc, acc[j]);
           } else {

@@ -14,18 +14,17 @@ namespace sq {
 // sq_check_device_error.
 __device__ unsigned int g_error_word;
 constexpr unsigned kErrTimeout = 1u;
-// Wall-clock limit of one wait.
-constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+// Limit of one wait in SM clock cycles: about 2 s at the 1965 MHz boost clock
+// (longer at lower clocks).  The SM cycle counter is read in a few cycles;
+// the global nanosecond timer, read in every turn of a spin loop, kept the
+// XU pipe busy and made each wait end late.
+constexpr long long kWaitLimitCycles = 4000000000ll;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ unsigned long long globaltimer_ns() {
-  unsigned long long t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
+__device__ __forceinline__ long long sm_cycles() { return clock64(); }
 
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
@@ -72,21 +71,38 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 
 // Wait until the phase with the given parity has completed.  Returns false
 // if the wait gave up: either the CTA-wide abort flag was raised by another
-// role, or this wait exceeded kWaitLimitNs (then it raises the flag and the
-// device error word).
+// role, or this wait exceeded `limit` SM cycles (then it raises the flag and
+// the device error word).
 __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity,
-                                             volatile int* abort_flag) {
+                                             volatile int* abort_flag,
+                                             long long limit = kWaitLimitCycles) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
-  const unsigned long long t0 = globaltimer_ns();
+  const long long t0 = sm_cycles();
   for (;;) {
     if (mbar_try_wait(a, parity)) return true;
     if (*abort_flag) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (sm_cycles() - t0 > limit) {
       *abort_flag = 1;
       atomicOr(&g_error_word, kErrTimeout);
       return false;
     }
+  }
+}
+
+// Self-test of the timeout path: one thread waits on an mbarrier that nothing
+// arrives on, with a short limit; the wait gives up, raises the abort flag
+// and latches the device error word exactly as a GEMM role's wait would.  No
+// copy, MMA or tensor memory is involved, so the kernel simply returns.
+__global__ void wait_timeout_selftest_kernel(long long limit_cycles, int* gave_up) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+    const bool ok = wait_bounded(&bar, 0, &abort_flag, limit_cycles);
+    *gave_up = ok ? 0 : (abort_flag ? 1 : 2);
   }
 }
 
@@ -113,10 +129,10 @@ __device__ __forceinline__ bool elect_one() {
 // flight before the CTA exits.
 __device__ __forceinline__ bool wait_drain(uint64_t* bar, uint32_t parity) {
   const uint32_t a = smem_u32(bar);
-  const unsigned long long t0 = globaltimer_ns();
+  const long long t0 = sm_cycles();
   for (;;) {
     if (mbar_try_wait(a, parity)) return true;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (sm_cycles() - t0 > kWaitLimitCycles) {
       atomicOr(&g_error_word, kErrTimeout);
       return false;
     }
@@ -380,7 +396,16 @@ __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
                    : "memory");
 }
-// Arrive on an mbarrier of another CTA of the cluster (cluster address).
+// Arrive on an mbarrier of another CTA of the cluster (cluster address) with
+// the default (release, CTA-scope) semantics: enough to hand a tensor-memory
+// buffer back after tcgen05.fence::before_thread_sync, and it does not wait
+// for this thread's outstanding global loads the way a cluster-scope release
+// does.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+// Arrive on an mbarrier of another CTA of the cluster (cluster address),
+// releasing this thread's shared-memory writes at cluster scope.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
                : "memory");
@@ -398,7 +423,7 @@ __device__ __forceinline__ void st_cluster_v4(uint32_t cluster_addr, uint32_t a,
 __device__ __forceinline__ bool wait_bounded_cluster(uint64_t* bar, uint32_t parity,
                                                      volatile int* abort_flag) {
   const uint32_t a = smem_u32(bar);
-  const unsigned long long t0 = globaltimer_ns();
+  const long long t0 = sm_cycles();
   for (;;) {
     uint32_t ok;
     asm volatile(
@@ -410,7 +435,7 @@ __device__ __forceinline__ bool wait_bounded_cluster(uint64_t* bar, uint32_t par
         : "memory");
     if (ok) return true;
     if (*abort_flag) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (sm_cycles() - t0 > kWaitLimitCycles) {
       *abort_flag = 1;
       atomicOr(&g_error_word, kErrTimeout);
       return false;

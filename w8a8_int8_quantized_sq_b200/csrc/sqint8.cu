@@ -9,6 +9,8 @@
 #include "../../include/sqint8.h"
 #include "gemm.cuh"
 #include "gemm2.cuh"
+#include "gemm3.cuh"
+#include "peak.cuh"
 #include "quant.cuh"
 
 using namespace sq;
@@ -101,6 +103,7 @@ bool block_scaled(GemmKind k) { return k == GK_GS128 || k == GK_PG128 || k == GK
 
 struct GemmPlan {
   bool pair;  // CTA-pair kernel (256 x 256 tiles per cluster of two)
+  bool pair3; // block-scaled CTA-pair kernel (256 x 128 tiles, a K block at a time)
   bool swap;
   int bn;
   bool stream_k;
@@ -125,9 +128,11 @@ bool pair_enabled() {
 }
 
 // sq_set_overlap: GEMM launches become programmatic dependents of the
-// preceding kernel on the stream (they request weights before that kernel ends).
-std::atomic<int> g_overlap{0};
-bool overlap_on() { return g_overlap.load(std::memory_order_relaxed) != 0; }
+// preceding kernel on the stream (they request weights before that kernel
+// ends).  The setting belongs to the host thread that made it: calls from
+// other threads keep the default.
+thread_local int t_overlap = 0;
+bool overlap_on() { return t_overlap != 0; }
 
 GemmPlan plan_gemm(GemmKind kind, int64_t M, int64_t N, int64_t K, int sms) {
   GemmPlan p{};
@@ -158,6 +163,18 @@ GemmPlan plan_gemm(GemmKind kind, int64_t M, int64_t N, int64_t K, int sms) {
       p.grid = sms;
     }
     p.ws_bytes = kCounterBytes + static_cast<size_t>(p.grid) * 2 * 128 * p.bn * 4;
+  } else if ((kind == GK_GS128 || kind == GK_FP8BLK) && pair_enabled()) {
+    // gs128: A = weights (256 channels per pair tile), B = tokens (128);
+    // FP8: A = tokens (256), B = weights (128 channels = one weight block)
+    p.pair3 = true;
+    p.swap = kind == GK_GS128;
+    p.bn = 128;
+    p.tiles_r = static_cast<int>(((p.swap ? N : M) + 255) / 256);
+    p.tiles_c = static_cast<int>(((p.swap ? M : N) + 127) / 128);
+    p.stream_k = false;
+    p.total_iters = static_cast<long long>(p.tiles_r) * p.tiles_c * p.kb_total;
+    p.grid = 0;  // decided at launch from the active-cluster limit
+    p.ws_bytes = 0;
   } else if ((kind == GK_I8_SCALE || kind == GK_I8_I32 || kind == GK_BF16) && pair_enabled()) {
     p.pair = true;
     p.swap = false;
@@ -308,6 +325,42 @@ sq_status launch_gemm2(const CUtensorMap& a, const CUtensorMap& b, const GemmArg
   return launch_status();
 }
 
+template <class Cfg>
+sq_status launch_gemm3(const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& g,
+                       cudaStream_t st, bool pdl) {
+  const int smem = Cfg::smem_bytes();
+  static std::atomic<int> max_clusters[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SQ_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(Cfg::THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 2 : 1;
+  int mc = max_clusters[dev].load(std::memory_order_acquire);
+  if (mc <= 0) {
+    if (cudaFuncSetAttribute(gemm3_kernel<Cfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem) != cudaSuccess)
+      return SQ_ERR_CUDA;
+    cfg.gridDim = dim3(2);
+    if (cudaOccupancyMaxActiveClusters(&mc, gemm3_kernel<Cfg>, &cfg) != cudaSuccess || mc <= 0)
+      return SQ_ERR_CUDA;
+    max_clusters[dev].store(mc, std::memory_order_release);
+  }
+  const int clusters = g.num_tiles < mc ? g.num_tiles : mc;
+  cfg.gridDim = dim3(2 * clusters);
+  if (cudaLaunchKernelEx(&cfg, gemm3_kernel<Cfg>, a, b, g) != cudaSuccess) return SQ_ERR_CUDA;
+  return launch_status();
+}
+
 // act: q_a int8 [M,K] or x bf16 [M,K]; wt: q_w int8 [N,K] or bf16 [N,K].
 sq_status run_gemm(GemmKind kind, const void* act, const void* wt, const float* s_tok,
                    const float* s_ch, const float* s_blk, void* out, int64_t M, int64_t N,
@@ -336,8 +389,9 @@ sq_status run_gemm(GemmKind kind, const void* act, const void* wt, const float* 
   } else if (!make_map(&ta, a_ptr, bf16, static_cast<uint64_t>(K), a_rows, kbe, 128)) {
     return SQ_ERR_CUDA;
   }
-  // the pair kernel stages 128 of the tile's 256 weight rows in each CTA
-  if (!make_map(&tb, b_ptr, bf16, static_cast<uint64_t>(K), b_rows, kbe, p.pair ? 128 : p.bn))
+  // the pair kernels stage half of the tile's B rows in each CTA
+  if (!make_map(&tb, b_ptr, bf16, static_cast<uint64_t>(K), b_rows, kbe,
+                p.pair ? 128 : (p.pair3 ? 64 : p.bn)))
     return SQ_ERR_CUDA;
 
   GemmArgs g{};
@@ -361,6 +415,10 @@ sq_status run_gemm(GemmKind kind, const void* act, const void* wt, const float* 
                     : nullptr;
   g.csplit = p.csplit;
 
+  if (p.pair3) {
+    if (kind == GK_GS128) return launch_gemm3<Gemm3Cfg<EPI_GS128>>(ta, tb, g, st, pdl);
+    return launch_gemm3<Gemm3Cfg<EPI_FP8BLK>>(ta, tb, g, st, pdl);
+  }
   if (p.pair) {
     if (kind == GK_I8_SCALE) return launch_gemm2<Gemm2Cfg<EPI_SCALE, 6>>(ta, tb, g, st, pdl);
     if (kind == GK_BF16)
@@ -624,6 +682,12 @@ sq_status sq_describe_plan(int op, int64_t M, int64_t N, int64_t K, int sms,
     r.tile_m = 256;
     r.tile_n = 256;
     r.splits = 1;
+  } else if (p.pair3) {
+    r.kernel = 4;
+    r.grid = 2 * (tiles < sms / 2 ? tiles : sms / 2);
+    r.tile_m = p.swap ? 128 : 256;
+    r.tile_n = p.swap ? 256 : 128;
+    r.splits = 1;
   } else if (!p.swap) {
     r.kernel = 1;
     r.grid = p.grid;
@@ -863,9 +927,52 @@ sq_status w8a16_group_mm(const void* x_bf16, const int8_t* q_w, const float* s_g
                   w_off, st);
 }
 
+sq_status sq_mma_peak(int kind, int iters, void* stream, double* ops_per_launch) {
+  if (!ops_per_launch) return SQ_ERR_NULL;
+  if (kind < 0 || kind > 2 || iters < 2 || iters > (1 << 24)) return SQ_ERR_SHAPE;
+  const int sms = num_sms();
+  if (sms < 2) return SQ_ERR_CUDA;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SQ_ERR_CUDA;
+  const int smem = 32768 + 1024;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  auto kern = kind == PEAK_I8 ? mma_peak_kernel<PEAK_I8>
+              : kind == PEAK_F8 ? mma_peak_kernel<PEAK_F8> : mma_peak_kernel<PEAK_BF16>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return SQ_ERR_CUDA;
+  cfg.gridDim = dim3(2);
+  int mc = 0;
+  if (cudaOccupancyMaxActiveClusters(&mc, kern, &cfg) != cudaSuccess || mc <= 0) return SQ_ERR_CUDA;
+  const int clusters = mc < sms / 2 ? mc : sms / 2;  // one pair per two SMs, all resident
+  cfg.gridDim = dim3(2 * clusters);
+  if (cudaLaunchKernelEx(&cfg, kern, iters) != cudaSuccess) return SQ_ERR_CUDA;
+  // M = 256, N = 256 and K = 32 (8-bit) or 16 (bf16) elements per MMA; 2 ops per MAC
+  const double k = kind == PEAK_BF16 ? 16.0 : 32.0;
+  *ops_per_launch = 2.0 * 256.0 * 256.0 * k * iters * clusters;
+  return launch_status();
+}
+
 sq_status sq_set_overlap(int enable) {
-  g_overlap.store(enable ? 1 : 0, std::memory_order_relaxed);
+  t_overlap = enable ? 1 : 0;
   return SQ_OK;
+}
+
+sq_status sq_selftest_wait_timeout(int64_t limit_cycles, int* gave_up, void* stream) {
+  if (!gave_up) return SQ_ERR_NULL;
+  if (limit_cycles <= 0 || limit_cycles > kWaitLimitCycles) return SQ_ERR_SHAPE;
+  wait_timeout_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_cycles,
+                                                                               gave_up);
+  return launch_status();
 }
 
 sq_status sq_check_device_error(int reset) {
