@@ -65,6 +65,9 @@ def test_block_scaled_pairs_and_large_m_w8a16():
     # FP8 blocks: tokens as A, 256 tokens x 128 channels (one weight block)
     p = plan(sq.OP_FP8BLK, 2048, 5120, 5120)
     assert (p["kernel"], p["tile_m"], p["tile_n"]) == (4, 256, 128)
+    # enough tiles for three waves of SM pairs: 256-wide B tiles
+    assert (plan(GS128, 8192, 34816, 5120)["tile_m"], plan(GS128, 8192, 34816, 5120)["tile_n"]) == (256, 256)
+    assert plan(sq.OP_FP8BLK, 8192, 34816, 5120)["tile_n"] == 256
     # per-group activations x gs128 weights: one CTA per 128 x 128 tile
     p = plan(sq.OP_PG128, 2048, 5120, 5120)
     assert (p["kernel"], p["tile_m"], p["tile_n"], p["grid"]) == (1, 128, 128, B200_SMS)

@@ -362,22 +362,27 @@ def set_overlap(enable: bool) -> None:
 PEAK_I8, PEAK_F8, PEAK_BF16 = 0, 1, 2
 
 
-def mma_peak(kind: int = PEAK_I8, iters: int = 8192, device=None) -> float:
+def mma_peak(kind: int = PEAK_I8, iters: int = 8192, launches: int = 4, device=None) -> float:
     """Measured dense tensor throughput (tera-ops/s) of the current device
-    for one MMA kind: sq_mma_peak launched on the current stream and timed
-    with CUDA events on that stream (best of three launches after a warm-up)."""
+    for one MMA kind: sq_mma_peak launched `launches` times back to back on
+    the current stream, each timed with CUDA events on that stream.  Short
+    launches (the default) give the burst rate, the best of all but the
+    first; long ones (iters ~ 2^21, about 0.3 s each) the rate under the power
+    cap, the mean of the second half of the launches."""
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
     ops = ctypes.c_double(0.0)
-    best = 0.0
-    for i in range(4):
+    rates = []
+    for i in range(launches):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
         _check("sq_mma_peak", lib().sq_mma_peak(kind, iters, _stream(dev), ctypes.byref(ops)))
         b.record()
         b.synchronize()
-        if i > 0:
-            best = max(best, ops.value / (a.elapsed_time(b) * 1e-3) / 1e12)
-    return best
+        rates.append(ops.value / (a.elapsed_time(b) * 1e-3) / 1e12)
+    if iters <= 65536:
+        return max(rates[1:]) if len(rates) > 1 else rates[0]
+    tail = rates[len(rates) // 2:]
+    return sum(tail) / len(tail)
 
 
 def selftest_wait_timeout(limit_cycles: int = 2_000_000, device=None) -> int:

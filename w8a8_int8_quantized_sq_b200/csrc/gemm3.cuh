@@ -56,22 +56,35 @@ __device__ __forceinline__ void mma_f8_pair(uint32_t d_tmem, uint64_t a, uint64_
       : "memory");
 }
 
-template <int EPI_>
+// Store 16 columns of one value to this warp's 32 tensor-memory lanes (no wait).
+__device__ __forceinline__ void tmem_st16_const(uint32_t taddr, uint32_t v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(taddr),
+      "r"(v)
+      : "memory");
+}
+
+// BN_: MMA N, the pair tile's B rows (128 or 256).  BIAS_: the int32
+// accumulators start at 0x4B400000 (gs128 only), see above.
+template <int EPI_, int BN_, bool BIAS_>
 struct Gemm3Cfg {
   static constexpr int EPI = EPI_;
   static constexpr bool F8 = EPI == EPI_FP8BLK;
   static constexpr bool SWAP = EPI == EPI_GS128;  // A = weights for gs128
+  static constexpr bool BIAS = BIAS_;
   static constexpr int BM = 128;         // A rows per CTA (256 per pair)
-  static constexpr int BN = 128;         // MMA N: B rows per pair tile
-  static constexpr int BN_CTA = 64;      // B rows staged by each CTA
+  static constexpr int BN = BN_;         // MMA N: B rows per pair tile
+  static constexpr int BN_CTA = BN / 2;  // B rows staged by each CTA
   static constexpr int A_BYTES = BM * 128;
   static constexpr int B_BYTES = BN_CTA * 128;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = 8;
-  static constexpr int NE = 8;           // epilogue warps
-  static constexpr int CPT = BN / (NE / 4);  // accumulator columns per epilogue thread
+  static constexpr int STAGES = BN == 256 ? 6 : 8;
+  static constexpr int NE = BN == 256 ? 16 : 8;   // epilogue warps
+  static constexpr int CPT = BN / (NE / 4);       // accumulator columns per epilogue thread
+  static constexpr int CHUNK = 16;                // columns per tensor-memory load
   static constexpr int THREADS = 64 + NE * 32;
-  static constexpr int NACC = 4;
+  static constexpr int NACC = 512 / BN;           // accumulator buffers
   static constexpr int TMEM_COLS = 512;
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = STAGES * A_BYTES;
@@ -80,6 +93,8 @@ struct Gemm3Cfg {
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int smem_bytes() { return 1024 + OFF_MISC + 16; }
   static_assert(EPI == EPI_GS128 || EPI == EPI_FP8BLK, "pair block-scaled epilogues");
+  static_assert(!BIAS || !F8, "the bias is an int32 bit pattern");
+  static_assert(CPT == 64 && CPT % CHUNK == 0, "epilogue layout");
 };
 
 template <class Cfg>
@@ -180,7 +195,10 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       for (int t = cluster; ok && t < g.num_tiles; t += nclusters) {
         for (int kb = 0; kb < g.kb_total; ++kb, ++local) {
           const uint32_t p = local % NACC, u = local / NACC;
-          if (!warp_wait_bounded(tempty + p, (u & 1u) ^ 1u, abort_flag)) { ok = false; break; }
+          // with the bias a buffer is free once the epilogue has re-armed it
+          // (the first time before any MMA); without it a buffer starts free
+          const uint32_t par = Cfg::BIAS ? (u & 1u) : ((u & 1u) ^ 1u);
+          if (!warp_wait_bounded(tempty + p, par, abort_flag)) { ok = false; break; }
           if (!warp_wait_bounded(full + stage, phase, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = smem_u32(smA + stage * Cfg::A_BYTES);
@@ -188,13 +206,14 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           const uint32_t d = tmem + p * BN;
           if (elect_one()) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {  // a fresh accumulator per K block
+            for (int k = 0; k < 4; ++k) {  // a fresh accumulator (or the bias) per K block
+              const uint32_t acc = (Cfg::BIAS || k > 0) ? 1u : 0u;
               if constexpr (Cfg::F8)
                 mma_f8_pair(d, smem_desc_sw128(sa + k * 32), smem_desc_sw128(sb + k * 32), idesc,
-                            k > 0 ? 1u : 0u);
+                            acc);
               else
                 mma_i8_pair(d, smem_desc_sw128(sa + k * 32), smem_desc_sw128(sb + k * 32), idesc,
-                            k > 0 ? 1u : 0u);
+                            acc);
             }
             mma_commit_pair_both(empty + stage);
             mma_commit_pair_both(tfull + p);
@@ -213,13 +232,15 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     // ------------------------------------------------------------ epilogue
     griddep_wait();
     const int ew = warp - 2;
-    constexpr int CPT = Cfg::CPT;
+    constexpr int CPT = Cfg::CPT, CHUNK = Cfg::CHUNK;
     const int q = warp & 3;                 // tensor-memory lane quadrant
     const int col0 = (ew >> 2) * CPT;       // this thread's accumulator columns
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16);
     const uint32_t tempty_leader = mapa_shared(smem_u32(tempty), 0);
     const int kbt = g.kb_total;
+    constexpr uint32_t kBias = 0x4B400000u;  // bits of 1.5 * 2^23
     auto release = [&](uint32_t p) {
+      if constexpr (Cfg::BIAS) tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
@@ -227,6 +248,14 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         else mbar_arrive_remote(tempty_leader + p * 8);
       }
     };
+    if constexpr (Cfg::BIAS) {
+      // arm every buffer with the bias before the first MMA
+      for (int p = 0; p < NACC; ++p) {
+#pragma unroll
+        for (int c = 0; c < CPT; c += CHUNK) tmem_st16_const(lane_base + p * BN + col0 + c, kBias);
+        release(p);
+      }
+    }
     uint32_t local = 0;
     bool ok = true;
     for (int t = cluster; ok && t < g.num_tiles; t += nclusters) {
@@ -235,63 +264,76 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       // or a token (FP8)
       const int arow = rt * 2 * Cfg::BM + static_cast<int>(rank) * Cfg::BM + q * 32 + lane;
       const bool row_ok = arow < (Cfg::SWAP ? g.N : g.M);
+      const int cbase = ct * BN + col0;     // this thread's first B row (token or channel)
       auto scale_of = [&](int kb) -> float {
         if constexpr (Cfg::SWAP) {
           return row_ok ? __ldg(g.s_blk + static_cast<size_t>(arow) * kbt + kb) : 0.0f;
         } else {
+          // the thread's 64 channels lie in one 128-channel weight block
           const float sa = row_ok ? __ldg(g.s_a + static_cast<size_t>(arow) * kbt + kb) : 0.0f;
-          return __fmul_rn(sa, __ldg(g.s_blk + static_cast<size_t>(ct) * kbt + kb));
+          const float sw = cbase < g.N ? __ldg(g.s_blk + static_cast<size_t>(cbase >> 7) * kbt + kb)
+                                       : 0.0f;
+          return __fmul_rn(sa, sw);
         }
       };
       float acc[CPT];
 #pragma unroll
       for (int j = 0; j < CPT; ++j) acc[j] = 0.0f;
-      // scales two K blocks ahead; each load is issued after the buffer
-      // release, so the release never waits for it
-      float sc = scale_of(0);
-      float sc1 = kbt > 1 ? scale_of(1) : 0.0f;
-      for (int kb = 0; kb < kbt; ++kb, ++local) {
+      // One K block.  Its scale s was loaded two K blocks earlier; the load
+      // for two K blocks later overwrites s after its last use.  (A rotating
+      // three-register prefetch made each K block wait for the load it had
+      // just issued: moving a register whose load is outstanding stalls.)
+      auto kblock = [&](int kb, float& s) {
         const uint32_t p = local % NACC, u = local / NACC;
-        if (!warp_wait_bounded(tfull + p, u & 1u, abort_flag)) { ok = false; break; }
+        ++local;
+        if (!ok) return;
+        if (!warp_wait_bounded(tfull + p, u & 1u, abort_flag)) { ok = false; return; }
         tc_fence_after();
-        uint32_t v[CPT];
-        tmem_ld64(lane_base + p * BN + col0, v);
-        release(p);
-        const float sc2 = kb + 2 < kbt ? scale_of(kb + 2) : 0.0f;
 #pragma unroll
-        for (int j = 0; j < CPT; ++j) {
-          // FP8: the fp32 partial; gs128: the exact f32(P)
-          const float f = Cfg::F8 ? __uint_as_float(v[j])
-                                  : __fsub_rn(__uint_as_float(v[j] + 0x4B400000u), 12582912.0f);
-          acc[j] = __fmaf_rn(f, sc, acc[j]);
+        for (int c = 0; c < CPT; c += CHUNK) {
+          uint32_t v[CHUNK];
+          tmem_ld16(lane_base + p * BN + col0 + c, v);
+          if constexpr (Cfg::BIAS) tmem_st16_const(lane_base + p * BN + col0 + c, kBias);
+          if (c + CHUNK == CPT) release(p);  // the whole K block is in registers or consumed
+#pragma unroll
+          for (int j = 0; j < CHUNK; ++j) {
+            float f;
+            if constexpr (Cfg::F8) f = __uint_as_float(v[j]);                 // fp32 partial
+            else if constexpr (Cfg::BIAS) f = __fsub_rn(__uint_as_float(v[j]), 12582912.0f);
+            else f = __fsub_rn(__uint_as_float(v[j] + kBias), 12582912.0f);  // exact f32(P)
+            acc[c + j] = __fmaf_rn(f, s, acc[c + j]);
+          }
         }
-        sc = sc1;
-        sc1 = sc2;
+        if (kb + 2 < kbt) s = scale_of(kb + 2);
+      };
+      float sa = scale_of(0);
+      float sb = kbt > 1 ? scale_of(1) : 0.0f;
+      for (int kb = 0; kb < kbt; kb += 2) {
+        kblock(kb, sa);
+        if (kb + 1 < kbt) kblock(kb + 1, sb);
       }
       if (!ok) break;
       // the tile's outputs
       __nv_bfloat16* out = static_cast<__nv_bfloat16*>(g.out);
       if constexpr (Cfg::SWAP) {
-        // lane = channel n, columns = tokens m
-        // lane j fetches the token scales of columns j and 32 + j (coalesced
-        // loads); the store loop takes them from that lane
-        static_assert(CPT == 64, "two token scales per lane");
-        const int m0 = ct * BN + col0;
-        const float st_lo = m0 + lane < g.M ? __ldg(g.s_tok + m0 + lane) : 0.0f;
-        const float st_hi = m0 + 32 + lane < g.M ? __ldg(g.s_tok + m0 + 32 + lane) : 0.0f;
-        __nv_bfloat16* o = out + static_cast<size_t>(m0) * g.N + arow;  // column j: o + j * N
+        // lane = channel n, columns = tokens m; lane j fetches the token
+        // scales of columns j and 32 + j (coalesced) and the stores take them
+        // from that lane
+        const float st_lo = cbase + lane < g.M ? __ldg(g.s_tok + cbase + lane) : 0.0f;
+        const float st_hi = cbase + 32 + lane < g.M ? __ldg(g.s_tok + cbase + 32 + lane) : 0.0f;
+        __nv_bfloat16* o = out + static_cast<size_t>(cbase) * g.N + arow;  // column j: o + j * N
 #pragma unroll
         for (int j = 0; j < CPT; ++j, o += g.N) {
           const float st = __shfl_sync(0xffffffffu, j < 32 ? st_lo : st_hi, j & 31);
-          if (row_ok && m0 + j < g.M) *o = __float2bfloat16_rn(__fmul_rn(acc[j], st));
+          if (row_ok && cbase + j < g.M) *o = __float2bfloat16_rn(__fmul_rn(acc[j], st));
         }
       } else {
-        // lane = token m, columns = channels n (one weight block)
+        // lane = token m, columns = channels n
         if (row_ok) {
           __nv_bfloat16* orow = out + static_cast<size_t>(arow) * g.N;
 #pragma unroll
           for (int j = 0; j < CPT; j += 8) {
-            const int n = ct * BN + col0 + j;
+            const int n = cbase + j;
             if (n + 8 <= g.N)
               *reinterpret_cast<uint4*>(orow + n) =
                   make_uint4(pack_bf16x2(acc[j], acc[j + 1]), pack_bf16x2(acc[j + 2], acc[j + 3]),

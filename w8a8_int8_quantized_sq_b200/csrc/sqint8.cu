@@ -127,6 +127,24 @@ bool pair_enabled() {
   return on;
 }
 
+// Width of the block-scaled pair tiles' MMA N (the B rows of a pair tile).
+// 256-wide tiles halve the accumulator round trips per multiply-add, but a
+// shape with fewer than three waves of them over the SM pairs loses more to
+// the partly filled last wave: M=8192 N=34816 K=5120 measured 2.46 ms (gs128)
+// and 1.82 ms (FP8) at 256 against 2.64 and 2.06 at 128; M=2048 N=5120
+// K=5120 measured 110 / 93 us at 128 against 120 / 97 at 256.
+// SQ_BLK_PAIR_N=128 or 256 overrides the choice (for comparisons).
+int blk_pair_bn(int64_t rows256, int64_t cols, int sms) {
+  static const int forced = [] {
+    const char* e = getenv("SQ_BLK_PAIR_N");
+    if (!e) return 0;
+    return e[0] == '1' ? 128 : (e[0] == '2' ? 256 : 0);
+  }();
+  if (forced) return forced;
+  const int64_t tiles256 = ((rows256 + 255) / 256) * ((cols + 255) / 256);
+  return tiles256 < 3 * (sms / 2) ? 128 : 256;
+}
+
 // sq_set_overlap: GEMM launches become programmatic dependents of the
 // preceding kernel on the stream (they request weights before that kernel
 // ends).  The setting belongs to the host thread that made it: calls from
@@ -168,9 +186,9 @@ GemmPlan plan_gemm(GemmKind kind, int64_t M, int64_t N, int64_t K, int sms) {
     // FP8: A = tokens (256), B = weights (128 channels = one weight block)
     p.pair3 = true;
     p.swap = kind == GK_GS128;
-    p.bn = 128;
+    p.bn = blk_pair_bn(p.swap ? N : M, p.swap ? M : N, sms);
     p.tiles_r = static_cast<int>(((p.swap ? N : M) + 255) / 256);
-    p.tiles_c = static_cast<int>(((p.swap ? M : N) + 127) / 128);
+    p.tiles_c = static_cast<int>(((p.swap ? M : N) + p.bn - 1) / p.bn);
     p.stream_k = false;
     p.total_iters = static_cast<long long>(p.tiles_r) * p.tiles_c * p.kb_total;
     p.grid = 0;  // decided at launch from the active-cluster limit
@@ -391,7 +409,7 @@ sq_status run_gemm(GemmKind kind, const void* act, const void* wt, const float* 
   }
   // the pair kernels stage half of the tile's B rows in each CTA
   if (!make_map(&tb, b_ptr, bf16, static_cast<uint64_t>(K), b_rows, kbe,
-                p.pair ? 128 : (p.pair3 ? 64 : p.bn)))
+                p.pair ? 128 : (p.pair3 ? p.bn / 2 : p.bn)))
     return SQ_ERR_CUDA;
 
   GemmArgs g{};
@@ -416,8 +434,12 @@ sq_status run_gemm(GemmKind kind, const void* act, const void* wt, const float* 
   g.csplit = p.csplit;
 
   if (p.pair3) {
-    if (kind == GK_GS128) return launch_gemm3<Gemm3Cfg<EPI_GS128>>(ta, tb, g, st, pdl);
-    return launch_gemm3<Gemm3Cfg<EPI_FP8BLK>>(ta, tb, g, st, pdl);
+    if (p.bn == 256) {
+      if (kind == GK_GS128) return launch_gemm3<Gemm3Cfg<EPI_GS128, 256, true>>(ta, tb, g, st, pdl);
+      return launch_gemm3<Gemm3Cfg<EPI_FP8BLK, 256, false>>(ta, tb, g, st, pdl);
+    }
+    if (kind == GK_GS128) return launch_gemm3<Gemm3Cfg<EPI_GS128, 128, false>>(ta, tb, g, st, pdl);
+    return launch_gemm3<Gemm3Cfg<EPI_FP8BLK, 128, false>>(ta, tb, g, st, pdl);
   }
   if (p.pair) {
     if (kind == GK_I8_SCALE) return launch_gemm2<Gemm2Cfg<EPI_SCALE, 6>>(ta, tb, g, st, pdl);
@@ -685,8 +707,8 @@ sq_status sq_describe_plan(int op, int64_t M, int64_t N, int64_t K, int sms,
   } else if (p.pair3) {
     r.kernel = 4;
     r.grid = 2 * (tiles < sms / 2 ? tiles : sms / 2);
-    r.tile_m = p.swap ? 128 : 256;
-    r.tile_n = p.swap ? 256 : 128;
+    r.tile_m = p.swap ? p.bn : 256;
+    r.tile_n = p.swap ? 256 : p.bn;
     r.splits = 1;
   } else if (!p.swap) {
     r.kernel = 1;
