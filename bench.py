@@ -6,8 +6,13 @@ dynamic INT8 quantisation of X with the SmoothQuant 1/s fold, then the
 INT8 x INT8 GEMM with the fused per-token x per-channel BF16 epilogue, on the
 prefill workload M=8192 tokens, K=5120, N=34816 (fused gate/up shape).
 The printed metric is TOPS (2*M*N*K per step, quantisation included in the
-time).  The same run also measures the decode W8A8 shape, the gs128
-variant and the W8A16 (down_proj) variant at M = 1, 16, 8192.
+time), over a short burst of steps (`value`) and over two seconds of steps
+(`sustained`, under the power cap), with the device's INT8 tensor rate
+measured by the library's issue-rate probe for each.  The same run also
+measures the decode W8A8 shape, the gs128 variant, the W8A16 (down_proj)
+variant at M = 1, 16, 8192, and the next rows: fused RMSNorm quantisation,
+per-group INT8 / FP8 activation quantisation, per-group x gs128 and FP8
+block GEMMs, and group-wise W8A16.
 
   python bench.py [--gpus N --steps K --warmup W] [--impl reference]
 
@@ -324,6 +329,13 @@ def main():
     y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     torch.cuda.synchronize()
 
+    # The dense INT8 (and FP8) tensor rate of this device, measured first,
+    # on a cool GPU, with the library's tcgen05 issue-rate probe (burst:
+    # about a millisecond per launch); 2 x the measured BF16 matmul is kept
+    # beside it for reference.
+    int8_probe = sq.mma_peak(sq.PEAK_I8)
+    fp8_probe = sq.mma_peak(sq.PEAK_F8)
+
     # One step = the whole layer through the fused entry point
     # (sq_w8a8_linear: quant, then the GEMM as a programmatic dependent).
     def step():
@@ -342,25 +354,6 @@ def main():
     barrier()
     clocks = sampler.result()
     total_s = max_over_ranks(start.elapsed_time(end) * 1e-3)
-
-    # Sustained: the same step back to back for at least two seconds (the
-    # short loop above is a burst that ends before the power cap settles).
-    sus_steps = max(args.steps, int(2.0 / max(total_s / args.steps, 1e-6)) + 1)
-    sampler = ClockSampler(local)
-    barrier()
-    sampler.start()
-    start.record()
-    for _ in range(sus_steps):
-        step()
-    end.record()
-    barrier()
-    sus_clocks = sampler.result()
-    sus_s = max_over_ranks(start.elapsed_time(end) * 1e-3)
-    sus_tops = whole_job_tops(2.0 * M * N * K, sus_steps, world, sus_s)
-    sustained = {"value": sus_tops, "unit": "TOPS", "steps": sus_steps, "seconds": sus_s,
-                 "ms_per_step": sus_s / sus_steps * 1e3, "clocks": sus_clocks,
-                 "tops_per_ghz": (sus_tops / (sus_clocks["sm_mhz"] / 1000.0)
-                                  if sus_clocks.get("sm_mhz") else None)}
 
     # The kernels on their own, live, same inputs: CUDA events around every
     # launch on the launching stream (the GEMM timing is the roofline's).
@@ -386,16 +379,35 @@ def main():
     del xs
     ops_step = 2.0 * M * N * K
     value = whole_job_tops(ops_step, args.steps, world, total_s)
-    # the dense INT8 (and FP8) tensor rate of this device, measured with the
-    # library's tcgen05 issue-rate probe; 2 x the measured BF16 matmul is kept
-    # beside it for reference
-    int8_probe = sq.mma_peak(sq.PEAK_I8)
-    fp8_probe = sq.mma_peak(sq.PEAK_F8)
     int8_proxy = peaks["bf16_tflops"] * INT8_PER_BF16
     int8_peak = int8_probe if int8_probe > 0 else int8_proxy
     peaks["int8_tops"] = int8_peak
     peaks["fp8_tops"] = fp8_probe if fp8_probe > 0 else int8_peak
     gemm_tops = ops_step / gemm_s / 1e12
+
+    # Sustained: the same step back to back for at least two seconds (the
+    # short loop above is a burst that ends before the power cap settles).
+    sus_steps = max(args.steps, int(2.0 / max(total_s / args.steps, 1e-6)) + 1)
+    sampler = ClockSampler(local)
+    barrier()
+    sampler.start()
+    start.record()
+    for _ in range(sus_steps):
+        step()
+    end.record()
+    barrier()
+    sus_clocks = sampler.result()
+    sus_s = max_over_ranks(start.elapsed_time(end) * 1e-3)
+    sus_tops = whole_job_tops(2.0 * M * N * K, sus_steps, world, sus_s)
+    sustained = {"value": sus_tops, "unit": "TOPS", "steps": sus_steps, "seconds": sus_s,
+                 "ms_per_step": sus_s / sus_steps * 1e3, "clocks": sus_clocks,
+                 "tops_per_ghz": (sus_tops / (sus_clocks["sm_mhz"] / 1000.0)
+                                  if sus_clocks.get("sm_mhz") else None)}
+    # the tensor rate under the same conditions: the probe run back to back
+    # for about two seconds right after
+    sus_probe = sq.mma_peak(sq.PEAK_I8, iters=1 << 21, launches=8)
+    sustained["int8_peak_sustained"] = sus_probe
+    sustained["frac_of_sustained_peak"] = sus_tops / sus_probe if sus_probe > 0 else None
 
     # ---------------- end to end through the public API, host buffers
     e2e_steps = max(3, min(args.steps, 10))
@@ -444,7 +456,6 @@ def main():
                                     "all SMs, burst)",
                      "peak_bf16x2": int8_proxy,
                      "frac_of_bf16x2": gemm_tops / int8_proxy,
-                     "frac_of_sustained": gemm_tops / (peaks["bf16_tflops_sustained"] * INT8_PER_BF16),
                      "traffic": gemm_traffic(),
                      "algorithmic_bytes": algo_bytes_w8a8(M, N, K)},
         "split_ms": {"quant": quant_s * 1e3, "gemm": gemm_s * 1e3,
@@ -460,6 +471,7 @@ def main():
     torch.cuda.empty_cache()
 
     line["measured_peaks"] = {"int8_tops": int8_probe, "fp8_tops": fp8_probe,
+                              "int8_tops_sustained": sustained["int8_peak_sustained"],
                               "hbm_gbs": peaks["hbm_gbs"], "bf16_tflops": peaks["bf16_tflops"]}
     if not args.no_variants:
         line["variants"] = variants(sq, inputs, dev, peaks) + variants_next(sq, inputs, dev, peaks)
