@@ -245,6 +245,53 @@ def oracle_sample(wl, target_s: float, max_rows: int = None):
     return rows, nt, run
 
 
+def oracle_other_configs(inputs):
+    """The CPU oracle timed once on each of the other workloads, in each
+    workload's own metric (a bounded row sample where the full workload would
+    take more than a few seconds; the sample is stated)."""
+    import oracle
+    out = []
+
+    def timed(fn):
+        t0 = time.perf_counter()
+        fn()
+        return time.perf_counter() - t0
+
+    for i in (0, 1):  # tiny and decode W8A8: quant + GEMM, all rows
+        wl = inputs.workload(i)
+        x, w = wl.make_x(), wl.make_w()
+        s, inv = oracle.smooth_factors(x, w)
+        q_w, s_ch = oracle.quant_weight(w, s)
+
+        def run():
+            q_a, s_tok = oracle.quant_per_token(x, inv)
+            oracle.w8a8_scaled_mm(q_a, s_tok, q_w, s_ch)
+        t = timed(run)
+        byt = algo_bytes_quant(wl.M, wl.K) + algo_bytes_w8a8(wl.M, wl.N, wl.K)
+        out.append({"workload": wl.name, "metric": "GB/s (quant + GEMM, algorithmic bytes)",
+                    "value": byt / t / 1e9, "unit": "GB/s", "seconds": t,
+                    "tops": 2.0 * wl.M * wl.N * wl.K / t / 1e12, "sample": "all rows"})
+    wl = inputs.workload(3)  # gs128: a row sample
+    x, w = wl.make_x(), wl.make_w()
+    q_w, s_blk = oracle.quant_weight(w, None, group=128)
+    rows = 256
+    q_a, s_tok = oracle.quant_per_token(x[:rows].contiguous(), None)
+    t = timed(lambda: oracle.gs128_mm(q_a, s_tok, q_w, s_blk))
+    out.append({"workload": wl.name, "metric": "TOPS (gs128 GEMM)",
+                "value": 2.0 * rows * wl.N * wl.K / t / 1e12, "unit": "TOPS", "seconds": t,
+                "sample": f"first {rows} of {wl.M} token rows, all N columns"})
+    wl = inputs.workload(4)  # W8A16 down_proj
+    w = wl.make_w()
+    q_w, s_ch = oracle.quant_weight(w, None)
+    for M in (1, 16):
+        x = wl.make_x(M)
+        t = timed(lambda: oracle.w8a16_mm(x, q_w, s_ch))
+        out.append({"workload": f"{wl.name}_M{M}", "metric": "GB/s (algorithmic bytes)",
+                    "value": algo_bytes_w8a16(M, wl.N, wl.K) / t / 1e9, "unit": "GB/s",
+                    "seconds": t, "sample": "all rows"})
+    return out
+
+
 def reference_arm(args, peaks):
     ws, rank, _ = dist_info()
     if rank != 0:
@@ -483,7 +530,8 @@ def main():
             "value": 2.0 * rows * N * K / t / 1e12, "unit": "TOPS", "cores": nt,
             "kind": "oracle", "seconds": t,
             "sample": f"first {rows} of {M} token rows of {wl.name} (oracle quant + GEMM + "
-                      "epilogue over all N columns)"}
+                      "epilogue over all N columns)",
+            "per_config": oracle_other_configs(inputs)}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
