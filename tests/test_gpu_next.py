@@ -257,3 +257,42 @@ def test_fp8_block_shapes(M, N, K):
     q_w, s_w = oracle.quant_fp8_block(w)
     _fp8_gemm_check(q_a, s_a, q_w, s_w, what=f"FP8 block M={M} K={K} N={N}")
     sq.check_device_error()
+
+
+# ------------------------------------------- 256-wide block-scaled pair tiles
+
+def test_block_scaled_wide_tiles_with_a_ragged_last_tile():
+    """M=8192, N=1920, K=256: enough tiles that the pair kernels take 256-wide
+    B tiles, and N % 256 = 128 leaves the last tile half filled (zero-filled
+    weight rows, guarded scales and stores).  gs128 bit-exact, FP8 within
+    its bound, on a row sample."""
+    M, N, K = 8192, 1920, 256
+    assert sq.describe_plan(sq.OP_GS128, M, N, K, 148)["tile_n"] == 256
+    assert sq.describe_plan(sq.OP_FP8BLK, M, N, K, 148)["tile_n"] == 256
+    x = inputs.gen_x(M, K, 96, inputs.XRecipe(col_count=3, col_factor=30.0, row_period=512,
+                                               row_width=4, row_factor=50.0))
+    w = inputs.gen_w(N, K, 96)
+    rng = np.random.default_rng(96)
+    rows = sorted({0, 255, 256, 8191} | set(rng.integers(0, M, 60).tolist()))
+    # gs128 (weights as the MMA's A operand)
+    q_a, s_tok = oracle.quant_per_token(x)
+    q_w, s_blk = oracle.quant_weight(w, None, group=128)
+    y = sq.w8a8_gs128_mm(q_a.cuda(), s_tok.cuda(), q_w.cuda(), s_blk.cuda()).cpu()
+    assert_same(y[rows], oracle.gs128_mm(q_a, s_tok, q_w, s_blk, rows=rows), "gs128 wide tiles")
+    # FP8 blocks (tokens as the MMA's A operand)
+    qf_a, sf_a = oracle.quant_fp8_per_group(x)
+    qf_w, sf_w = oracle.quant_fp8_block(w)
+    _fp8_gemm_check(qf_a, sf_a, qf_w, sf_w, rows=rows, what="FP8 block M=8192 K=256 N=1920 (rows)")
+    sq.check_device_error()
+
+
+def test_mma_peak_probe_is_plausible():
+    """The issue-rate probe behind the roofline denominators: dense INT8 and
+    FP8 rates between 1 and 6 POPS on a B200 (4.5 nominal), BF16 about half."""
+    i8 = sq.mma_peak(sq.PEAK_I8)
+    f8 = sq.mma_peak(sq.PEAK_F8)
+    bf = sq.mma_peak(sq.PEAK_BF16)
+    print(f"\nmeasured dense rates: INT8 {i8:.0f}, FP8 {f8:.0f}, BF16 {bf:.0f} TOPS")
+    assert 1000 < i8 < 6000 and 1000 < f8 < 6000
+    assert 0.35 < bf / i8 < 0.65
+    sq.check_device_error()
