@@ -6,12 +6,12 @@
 // Both promote every 128-wide K block separately: the K block's MMAs write a
 // fresh accumulator in tensor memory and the epilogue warps fold it into fp32
 // registers with that block's scale.  The pair tile is 256 MMA rows (128 in
-// each CTA's tensor memory) x 128 MMA columns; each CTA stages its own 128
-// A rows and 64 of the 128 B rows per K block (24 KB), so a CTA's shared
-// memory carries 6 KB of operands per 128 x 128 x 32 MMA step instead of the
-// 8 KB of a single-CTA 128 x 128 tile.  Tensor memory holds four 128-column
-// accumulators per CTA, so the MMA runs up to three K blocks ahead of the
-// epilogue.
+// each CTA's tensor memory) x BN MMA columns, BN = 128 or 256; each CTA
+// stages its own 128 A rows and BN / 2 of the B rows per K block.
+//   BN = 128: four 128-column accumulators per CTA, 8 epilogue warps.
+//   BN = 256: two 256-column accumulators, 16 epilogue warps (64 columns
+//          each, loaded 16 at a time to fit 96 registers).  The host picks it
+//          when the shape has at least three waves of 256-wide pair tiles.
 //
 // The operand roles are chosen so that each epilogue thread needs a single
 // scale per K block:
@@ -19,23 +19,28 @@
 //          n (its tensor-memory lane): acc = fmaf(f32(P), s_blk[n,kb], acc),
 //          and y = bf16(acc * s_tok[m]) at the end of the tile.
 //   FP8 (not swapped): A = tokens, B = weights.  A thread owns one token m
-//          and the tile's 128 channels are one weight block:
+//          and its 64 channels lie in one 128-channel weight block:
 //          acc = fmaf(P, f32(s_a[m,kb] * s_w[n/128,kb]), acc), y = bf16(acc).
 // The int32 partials of gs128 become fp32 exactly (|P| <= 128 * 127^2 <
-// 2^22: add the bits of 1.5 * 2^23, subtract 1.5 * 2^23), then one fmaf per
-// element: the oracle's sequence.
+// 2^22): the bits of 1.5 * 2^23 are added, then 1.5 * 2^23 is subtracted, and
+// one fmaf per element follows, the oracle's sequence.  With BN = 256 the
+// accumulators start at those bits (0x4B400000) and all MMAs of a K block
+// accumulate onto them, so the int32 result already is the fp32 pattern of
+// 1.5 * 2^23 + P; the epilogue re-arms the bias with a tensor-memory store.
 //
 // Pace: each K block's accumulator makes a round trip MMA -> commit ->
-// epilogue -> release -> MMA warp, and with 128-column MMAs (about 140 ns of
-// tensor work per K block) four buffers do not cover it.  A probe issuing the
-// same pair MMAs with a commit per K block and a wait four blocks back ran at
-// two thirds of the back-to-back rate; with 256-column MMAs and two buffers
-// it lost nothing.  Measured variants of this kernel: 16 epilogue warps with
-// the magic-number bias kept in tensor memory, and packed f32x2 promotion,
-// were both slower than this one.
+// epilogue -> release -> MMA warp.  A probe issuing the same pair MMAs with a
+// commit per K block and a wait four blocks back ran at two thirds of the
+// back-to-back rate with 128-column MMAs and lost nothing with 256-column MMAs
+// and two buffers.  Beyond that, promoting per K block moves 128 * BN * 4
+// bytes per CTA per K block out of tensor memory and costs two or three
+// instructions per element.  Measured variants that were slower: packed
+// f32x2 promotion; 16 epilogue warps on 128-wide tiles; a 256-thread barrier
+// per K block; a cluster-scope releasing arrive (it waited for the
+// outstanding scale loads); scale windows staged in shared memory.
 //
 // Roles per CTA: warp 0 TMA producer, warp 1 tensor-memory allocation (pair)
-// and, in the leader CTA, the MMA issuer, warps 2..9 epilogue (two per
+// and, in the leader CTA, the MMA issuer, the other warps epilogue (NE / 4 per
 // tensor-memory lane quadrant, 64 columns each).  No load uses multicast.
 #pragma once
 #include "gemm2.cuh"
