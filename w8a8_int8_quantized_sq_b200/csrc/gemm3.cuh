@@ -32,9 +32,11 @@
 // epilogue -> release -> MMA warp.  A probe issuing the same pair MMAs with a
 // commit per K block and a wait four blocks back ran at two thirds of the
 // back-to-back rate with 128-column MMAs and lost nothing with 256-column MMAs
-// and two buffers.  Beyond that, promoting per K block moves 128 * BN * 4
-// bytes per CTA per K block out of tensor memory and costs two or three
-// instructions per element.  Measured variants that were slower: packed
+// and two buffers.  Beyond that, a buffer goes back to the MMA only once every
+// epilogue warp of both CTAs has released it, and promotion costs two or
+// three instructions per element; tensor-memory loads (450 bytes per SM
+// clock and more from 16 warps, measured) are not the limit.  Measured
+// variants that were slower: packed
 // f32x2 promotion; 16 epilogue warps on 128-wide tiles; a 256-thread barrier
 // per K block; a cluster-scope releasing arrive (it waited for the
 // outstanding scale loads); scale windows staged in shared memory.
