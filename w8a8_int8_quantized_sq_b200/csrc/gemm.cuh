@@ -94,7 +94,7 @@ __host__ __device__ constexpr int pow2_at_least(int v) {
 // the tensor pipe waiting on each commit.  Keeping A out of shared
 // memory leaves 2 bytes of shared-memory traffic per weight byte instead of 6.
 template <bool I8_, int BN_, int STAGES_, bool SWAP_, int EPI_, bool CONV_ = false,
-          int RSTAGES_ = 0>
+          int RSTAGES_ = 0, int BRING_ = 65536>
 struct GemmCfg {
   static constexpr bool I8 = I8_;
   static constexpr int BN = BN_;
@@ -134,9 +134,10 @@ struct GemmCfg {
   static constexpr int SBLK_STRIDE = BN + 4;    // floats per K block in the staged s_blk
   // shared memory carve-up (offsets from a 1024-byte aligned base)
   static constexpr int A_SMEM_BYTES = CONV ? 0 : A_BYTES;  // CONV: A lives in TMEM
-  // CONV: the B tiles have their own ring of stages of RK tiles (64 KB), so
-  // their loads run ahead of the MMAs instead of following the A stages
-  static constexpr int BSTAGES = CONV ? (65536 / (RK * B_BYTES)) : STAGES;
+  // CONV: the B tiles have their own ring of stages of RK tiles (BRING_
+  // bytes), so their loads run ahead of the MMAs instead of following the A
+  // stages
+  static constexpr int BSTAGES = CONV ? (BRING_ / (RK * B_BYTES)) : STAGES;
   static constexpr int B_RING_BYTES = CONV ? BSTAGES * RK * B_BYTES : STAGES * B_BYTES;
   static constexpr int OFF_RAW = 0;
   static constexpr int OFF_A = OFF_RAW + RSTAGES * RAW_BYTES;
@@ -160,6 +161,7 @@ struct GemmCfg {
   static_assert(EPI != EPI_W16G || CONV, "group-scaled reconstruction happens on load");
   static_assert(!CONV || (RAW_BYTES % 1024 == 0 && B_BYTES % 16 == 0), "raw stage alignment");
   static_assert(!CONV || ACC_COLS + STAGES * RK * A_TMEM_COLS <= 512, "tensor memory A ring");
+  static_assert(!CONV || BSTAGES >= 2, "B ring");
 
   static_assert(TMEM_COLS <= 512, "tensor memory");
 };
@@ -504,63 +506,62 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                            : 0.0f;
           }
           if (!wait_bounded(raw_full + rs, rph, abort_flag)) { ok = false; break; }
-          // the A stage is free once the MMAs that read it are done
-          if (!wait_bounded(empty + cs, cph ^ 1u, abort_flag)) { ok = false; break; }
-          tc_fence_after();
           const uint8_t* raw = smRaw + rs * Cfg::RAW_BYTES;
           // raw row (128-byte swizzle): K block c is chunks 4(c&1)..4(c&1)+3 of
           // its box row, 16-byte chunk j at position j ^ (row & 7).  This
           // thread converts chunks 2*half, 2*half+1 (32 codes -> 32 bf16, two
           // per column, lower K in the low half) into TMEM columns 16*half ..
           // 16*half+15 of the K block's part of the A stage.
+          constexpr int CH = 2;
           auto chunk = [&](int c, int jj) {
             return *reinterpret_cast<const uint4*>(
                 raw + (c >> 1) * Cfg::RAW_BOX_BYTES + row * 128 +
                 (((4 * (c & 1) + 2 * half + jj) ^ (row & 7)) << 4));
           };
-          auto convert = [&](const uint4 w0, const uint4 w1, uint32_t slot) {
-            uint32_t o[16];
-            if constexpr (Cfg::EPI == EPI_W16G) {
-              const float sc = gsc[slot];
-              i8x4_scale_to_bf16x4(w0.x, sc, o[0], o[1]);
-              i8x4_scale_to_bf16x4(w0.y, sc, o[2], o[3]);
-              i8x4_scale_to_bf16x4(w0.z, sc, o[4], o[5]);
-              i8x4_scale_to_bf16x4(w0.w, sc, o[6], o[7]);
-              i8x4_scale_to_bf16x4(w1.x, sc, o[8], o[9]);
-              i8x4_scale_to_bf16x4(w1.y, sc, o[10], o[11]);
-              i8x4_scale_to_bf16x4(w1.z, sc, o[12], o[13]);
-              i8x4_scale_to_bf16x4(w1.w, sc, o[14], o[15]);
-            } else {
-              i8x4_to_bf16x4(w0.x, o[0], o[1]);
-              i8x4_to_bf16x4(w0.y, o[2], o[3]);
-              i8x4_to_bf16x4(w0.z, o[4], o[5]);
-              i8x4_to_bf16x4(w0.w, o[6], o[7]);
-              i8x4_to_bf16x4(w1.x, o[8], o[9]);
-              i8x4_to_bf16x4(w1.y, o[10], o[11]);
-              i8x4_to_bf16x4(w1.z, o[12], o[13]);
-              i8x4_to_bf16x4(w1.w, o[14], o[15]);
+          auto convert = [&](const uint4 (&wc)[CH], uint32_t slot) {
+            uint32_t o[8 * CH];
+#pragma unroll
+            for (int j = 0; j < CH; ++j) {
+              if constexpr (Cfg::EPI == EPI_W16G) {
+                const float sc = gsc[slot];
+                i8x4_scale_to_bf16x4(wc[j].x, sc, o[8 * j + 0], o[8 * j + 1]);
+                i8x4_scale_to_bf16x4(wc[j].y, sc, o[8 * j + 2], o[8 * j + 3]);
+                i8x4_scale_to_bf16x4(wc[j].z, sc, o[8 * j + 4], o[8 * j + 5]);
+                i8x4_scale_to_bf16x4(wc[j].w, sc, o[8 * j + 6], o[8 * j + 7]);
+              } else {
+                i8x4_to_bf16x4(wc[j].x, o[8 * j + 0], o[8 * j + 1]);
+                i8x4_to_bf16x4(wc[j].y, o[8 * j + 2], o[8 * j + 3]);
+                i8x4_to_bf16x4(wc[j].z, o[8 * j + 4], o[8 * j + 5]);
+                i8x4_to_bf16x4(wc[j].w, o[8 * j + 6], o[8 * j + 7]);
+              }
             }
             tmem_st16(a_lane + (cs * Cfg::RK + slot) * Cfg::A_TMEM_COLS + half * 16, o);
           };
-          if (n == Cfg::RK) {
-            uint4 w[Cfg::RK][2];
+          // The whole stage's codes go to registers first and the raw stage
+          // is released at once (the arrive orders this warp's loads before
+          // it), so the next weight load is in flight while this warp waits
+          // for its A stage and converts: a raw stage is held for the length
+          // of a shared-memory load, not of a conversion.
+          uint4 w[Cfg::RK][CH];
 #pragma unroll
-            for (int c = 0; c < Cfg::RK; ++c) {  // all loads first
-              w[c][0] = chunk(c, 0);
-              w[c][1] = chunk(c, 1);
+          for (int c = 0; c < Cfg::RK; ++c) {
+            if (c < n) {
+#pragma unroll
+              for (int j = 0; j < CH; ++j) w[c][j] = chunk(c, j);
             }
-#pragma unroll
-            for (int c = 0; c < Cfg::RK; ++c) convert(w[c][0], w[c][1], c);
-          } else {
-            for (int c = 0; c < n; ++c) convert(chunk(c, 0), chunk(c, 1), c);
           }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(raw_empty + rs);
+          // the A stage is free once the MMAs that read it are done
+          if (!wait_bounded(empty + cs, cph ^ 1u, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < Cfg::RK; ++c)
+            if (c < n) convert(w[c], c);
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) {
-            mbar_arrive(raw_empty + rs);
-            mbar_arrive(full + cs);
-          }
+          if (lane == 0) mbar_arrive(full + cs);
           if (++cs == STAGES) { cs = 0; cph ^= 1u; }
           if (++rs == Cfg::RSTAGES) { rs = 0; rph ^= 1u; }
         }
