@@ -94,7 +94,7 @@ __host__ __device__ constexpr int pow2_at_least(int v) {
 // the tensor pipe waiting on each commit.  Keeping A out of shared
 // memory leaves 2 bytes of shared-memory traffic per weight byte instead of 6.
 template <bool I8_, int BN_, int STAGES_, bool SWAP_, int EPI_, bool CONV_ = false,
-          int RSTAGES_ = 0, int BRING_ = 65536>
+          int RSTAGES_ = 0>
 struct GemmCfg {
   static constexpr bool I8 = I8_;
   static constexpr int BN = BN_;
@@ -134,10 +134,10 @@ struct GemmCfg {
   static constexpr int SBLK_STRIDE = BN + 4;    // floats per K block in the staged s_blk
   // shared memory carve-up (offsets from a 1024-byte aligned base)
   static constexpr int A_SMEM_BYTES = CONV ? 0 : A_BYTES;  // CONV: A lives in TMEM
-  // CONV: the B tiles have their own ring of stages of RK tiles (BRING_
-  // bytes), so their loads run ahead of the MMAs instead of following the A
-  // stages
-  static constexpr int BSTAGES = CONV ? (BRING_ / (RK * B_BYTES)) : STAGES;
+  // CONV: the B tiles have their own ring of stages of RK tiles (64 KB), so
+  // their loads run ahead of the MMAs instead of following the A stages (a
+  // 32 KB ring measured 2 us slower at 16 tokens)
+  static constexpr int BSTAGES = CONV ? (65536 / (RK * B_BYTES)) : STAGES;
   static constexpr int B_RING_BYTES = CONV ? BSTAGES * RK * B_BYTES : STAGES * B_BYTES;
   static constexpr int OFF_RAW = 0;
   static constexpr int OFF_A = OFF_RAW + RSTAGES * RAW_BYTES;
@@ -161,7 +161,6 @@ struct GemmCfg {
   static_assert(EPI != EPI_W16G || CONV, "group-scaled reconstruction happens on load");
   static_assert(!CONV || (RAW_BYTES % 1024 == 0 && B_BYTES % 16 == 0), "raw stage alignment");
   static_assert(!CONV || ACC_COLS + STAGES * RK * A_TMEM_COLS <= 512, "tensor memory A ring");
-  static_assert(!CONV || BSTAGES >= 2, "B ring");
 
   static_assert(TMEM_COLS <= 512, "tensor memory");
 };
@@ -214,7 +213,8 @@ struct SegIter {
 template <class Cfg>
 __device__ __forceinline__ void store_chunk(const GemmArgs& g, int rt, int ct, int rr, int c0,
                                             const uint32_t (&v)[Cfg::CW], uint64_t policy = 0,
-                                            const float* sc_pre = nullptr) {
+                                            const float* sc_pre = nullptr,
+                                            const float* st_pre = nullptr) {
   constexpr int CW = Cfg::CW;
   const int r = rt * Cfg::BM + rr;
   const int cb = ct * Cfg::BN + c0;
@@ -277,7 +277,7 @@ __device__ __forceinline__ void store_chunk(const GemmArgs& g, int rt, int ct, i
         if (m < g.M) {
           float f;
           if constexpr (Cfg::I8) {
-            const float st = g.s_tok ? __ldg(g.s_tok + m) : 1.0f;
+            const float st = st_pre ? st_pre[j] : (g.s_tok ? __ldg(g.s_tok + m) : 1.0f);
             f = __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(v[j])), st), sc);
           } else {
             f = __fmul_rn(__uint_as_float(v[j]), sc);
@@ -877,6 +877,16 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       uint32_t local = 0;
       const long long G = gridDim.x, T = g.total_iters;
       const int me = blockIdx.x;
+      // Swapped W8A8 tiles hold every token in one chunk (M <= BN): their
+      // token scales are read once here, not in the tail of each tile.
+      constexpr bool kPreTok =
+          Cfg::SWAP && Cfg::I8 && Cfg::EPI == EPI_SCALE && Cfg::CW == Cfg::BN;
+      float stok[kPreTok ? Cfg::BN : 1];
+      if constexpr (kPreTok) {
+#pragma unroll
+        for (int j = 0; j < Cfg::BN; ++j)
+          stok[j] = (g.s_tok && j < g.M) ? __ldg(g.s_tok + j) : 1.0f;
+      }
       while (it.next(g, s)) {
         const uint32_t a = local % NACC, u = local / NACC;
         const int rt = s.tile % g.tiles_r, ct = s.tile / g.tiles_r;
@@ -889,6 +899,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         }
         const float* scp =
             (Cfg::SWAP && (Cfg::EPI == EPI_SCALE || Cfg::EPI == EPI_W16G)) ? &sc_pre : nullptr;
+        // swapped W8A8 tiles of one chunk: the token scales in registers
+        const float* stp = kPreTok ? stok : nullptr;
         const bool w_ok = wait_bounded(tfull + a, u & 1u, abort_flag);
         if (named_bar_or(1, nthr, !w_ok)) break;
         tc_fence_after();
@@ -899,7 +911,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           for (int c = 0; c < BN; c += CW) {
             uint32_t v[CW];
             tmem_ld_acc<Cfg>(tb, c, nsub, v);
-            store_chunk<Cfg>(g, rt, ct, rr, c, v, 0, scp);
+            store_chunk<Cfg>(g, rt, ct, rr, c, v, 0, scp, stp);
           }
         } else if (g.csplit > 1) {
           // cluster split-K: the tile's K parts are the ranks of this cluster
@@ -941,7 +953,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                   }
                 }
               }
-              store_chunk<Cfg>(g, rt, ct, rr, c, v, 0, scp);
+              store_chunk<Cfg>(g, rt, ct, rr, c, v, 0, scp, stp);
             }
           }
         } else {
@@ -1015,7 +1027,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                   }
                 }
               }
-              store_chunk<Cfg>(g, rt, ct, rr, c, v, 0, scp);
+              store_chunk<Cfg>(g, rt, ct, rr, c, v, 0, scp, stp);
             }
           }
         }

@@ -468,7 +468,7 @@ sq_status run_gemm(GemmKind kind, const void* act, const void* wt, const float* 
       return launch_gemm<GemmCfg<true, 128, 4, false, EPI_FP8BLK>>(ta, tb, g, p.grid, st, pdl);
     case GK_W8A16G_CONV:
       if (p.bn == 16)
-        return launch_gemm<GemmCfg<false, 16, 3, true, EPI_W16G, true, 6, 32768>>(ta, tb, g, p.grid,
+        return launch_gemm<GemmCfg<false, 16, 3, true, EPI_W16G, true, 5>>(ta, tb, g, p.grid,
                                                                           st, pdl);
       return launch_gemm<GemmCfg<false, 32, 2, true, EPI_W16G, true, 5>>(ta, tb, g, p.grid, st,
                                                                         pdl);
@@ -478,7 +478,7 @@ sq_status run_gemm(GemmKind kind, const void* act, const void* wt, const float* 
       return launch_gemm<GemmCfg<false, 256, 4, false, EPI_SCALE>>(ta, tb, g, p.grid, st, pdl);
     case GK_W8A16_CONV:
       if (p.bn == 16)
-        return launch_gemm<GemmCfg<false, 16, 3, true, EPI_SCALE, true, 6, 32768>>(ta, tb, g, p.grid,
+        return launch_gemm<GemmCfg<false, 16, 3, true, EPI_SCALE, true, 5>>(ta, tb, g, p.grid,
                                                                            st, pdl);
       return launch_gemm<GemmCfg<false, 32, 2, true, EPI_SCALE, true, 5>>(ta, tb, g, p.grid, st,
                                                                          pdl);
