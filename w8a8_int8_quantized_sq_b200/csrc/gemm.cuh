@@ -83,11 +83,11 @@ __host__ __device__ constexpr int pow2_at_least(int v) {
 
 // CONV_ = true (the W8A16 dequant-on-load path): operand A arrives as int8
 // weight rows, RK K blocks per raw shared-memory stage (TMA, 128-byte
-// swizzle).  Eight converter warps expand a whole raw stage exactly to bf16
-// and write it straight into a ring of STAGES A tiles in tensor memory
-// (tcgen05.st; 32 columns of two bf16 per 128-lane row per K block), then wait
-// for their stores once and release the raw stage; the MMA reads A from tensor
-// memory.  A producer warp of its own loads the K blocks' B tiles into their
+// swizzle).  Eight converter warps copy a whole raw stage into registers and
+// release it, then expand it exactly to bf16 and write it straight into a
+// ring of STAGES A tiles in tensor memory (tcgen05.st; 32 columns of two bf16
+// per 128-lane row per K block) and wait for their stores once; the MMA reads
+// A from tensor memory.  A producer warp of its own loads the K blocks' B tiles into their
 // own shared-memory ring.  Everything moves in groups of RK K blocks (one raw
 // stage, one A stage, one B stage): one hand-off and one tcgen05.commit per
 // 4 x RK MMAs, because short N = 16 MMAs committed one K block at a time keep
