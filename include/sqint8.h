@@ -109,9 +109,18 @@ sq_status w8a8_gs128_mm(const int8_t* q_a, const float* s_tok, const int8_t* q_w
  * [N,K], s_ch fp32 [N]; y = bf16_rne(s_ch[n] * sum_k x[m,k] * q_w[n,k]).
  * The int8 -> bf16 weight conversion is exact and the scale is applied in
  * the fp32 epilogue; products are exact and accumulate in fp32 (the order
- * of the fp32 sum is the kernel's).  Workspace (SQ_OP_W8A16) holds split-K
- * partials for small M and the converted BF16 weights for large M; the
- * zero-fill rule of w8a8_scaled_mm applies. */
+ * of the fp32 sum is the kernel's).
+ * M = 1 (K <= 30720) runs as a matrix-vector product on the CUDA cores in
+ * exact integer arithmetic: the token becomes v = rint(x * 2^sh), |v| < 2^31
+ * (sh from the exponent of max|x|; values more than 23 binades below the
+ * largest are rounded to the nearest 2^-sh), the dot products with the codes
+ * are exact (dp4a over the four bytes of v, combined in int64), and
+ * y = bf16_rne(fp64(sum) * s_ch * 2^-sh).  A token holding inf or NaN has
+ * no such image: every output of the call is then NaN.  Other small M
+ * convert the weights on load into the tensor cores.
+ * Workspace (SQ_OP_W8A16) holds split-K partials for small M (unused at
+ * M = 1) and the converted BF16 weights for large M; the zero-fill rule of
+ * w8a8_scaled_mm applies. */
 sq_status w8a16_mm(const void* x_bf16, const int8_t* q_w, const float* s_ch, void* y_bf16,
                    int64_t M, int64_t N, int64_t K, void* workspace, size_t ws_bytes,
                    void* stream);
@@ -262,7 +271,8 @@ sq_status sq_set_overlap(int enable);
  * thread-block cluster (a call falls back to 2 when the device cannot hold
  * every cluster at once or the parts do not fit in shared memory),
  * 4 = block-scaled CTA pairs (gs128: 128 tokens x 256 channels, FP8 blocks:
- * 256 tokens x 128 channels per pair tile).
+ * 256 tokens x 128 channels per pair tile), 5 = W8A16 with one token on the
+ * CUDA cores (a matrix-vector product, tile_n = most rows one CTA owns).
  * tile_m x tile_n: tokens x output channels per tile.  grid: CTAs (for
  * kernel 0 an upper bound: the launch takes the active-cluster limit).
  * splits: K parts per tile when every CTA owns one part of one tile, 0 when

@@ -197,7 +197,9 @@ def _check_w8a16(x, q_w, s_ch, rows=None):
     ref, mag = oracle.w8a16_mm(x, q_w, s_ch, rows=rows, with_bound=True)
     K = x.shape[1]
     # fp32 accumulation: at most K/16 tensor-core steps plus the split-K
-    # combination, each adding at most 2^-22 of the magnitude sum.
+    # combination, each adding at most 2^-22 of the magnitude sum.  One token
+    # runs as an exact integer dot product on a fixed-point image of the
+    # token (checked to 1 ulp in test_w8a16_single_token_*), well inside it.
     gamma = (K / 16 + 8) * 2.0 ** -22
     diff = (y.double() - ref.double()).abs()
     ulp = bf16_ulp(ref)
@@ -230,12 +232,72 @@ def test_w8a16_prefill_every_row_tile():
 
 
 @pytest.mark.parametrize("M,N,K", [(3, 144, 256), (17, 144, 384), (32, 256, 1280),
-                                   (8, 5120, 5120), (33, 256, 640)])
+                                   (8, 5120, 5120), (33, 256, 640),
+                                   # one token: matrix-vector kernel (fewer rows than
+                                   # SMs, ragged rows per CTA, partly idle warps, the
+                                   # widest block) and the tensor-core fallback past it
+                                   (1, 16, 128), (1, 144, 384), (1, 4096, 17408),
+                                   (1, 65536, 1024), (1, 144, 30720), (1, 272, 30848)])
 def test_w8a16_shapes(M, N, K):
     x = inputs.gen_x(M, K, 5)
     q_w = torch.randint(-127, 128, (N, K), dtype=torch.int8)
     s_ch = torch.rand(N) * 1e-3 + 1e-5
     _check_w8a16(x, q_w, s_ch)
+
+
+def _single_token(x, q_w, s_ch):
+    """One token: the matrix-vector kernel's sum is exact, so y is within
+    1 bf16 ulp of the oracle everywhere (the oracle's fp64 sum and one
+    rounding; both round sum * s_ch once, the kernel from the exact sum)."""
+    y = sq.w8a16_mm(x.cuda(), q_w.cuda(), s_ch.cuda()).cpu()
+    ref = oracle.w8a16_mm(x, q_w, s_ch)
+    diff = (y.double() - ref.double()).abs()
+    assert torch.all(diff <= bf16_ulp(ref)), float((diff / bf16_ulp(ref)).max())
+    differ = int((y.view(torch.int16) != ref.view(torch.int16)).sum())
+    print(f"\nW8A16 one token K={x.shape[1]} N={q_w.shape[0]}: {differ} of {y.numel()} "
+          "outputs differ from the oracle (none beyond 1 ulp)")
+    return y, ref
+
+
+@pytest.mark.parametrize("N,K", [(5120, 17408), (144, 384), (4096, 17408), (65536, 1024),
+                                 (144, 30720)])
+def test_w8a16_single_token_exact(N, K):
+    x = inputs.gen_x(1, K, 7)
+    g = torch.Generator().manual_seed(N + K)
+    q_w = torch.randint(-127, 128, (N, K), dtype=torch.int8, generator=g)
+    s_ch = torch.rand(N, generator=g) * 1e-3 + 1e-5
+    _single_token(x, q_w, s_ch)
+
+
+def test_w8a16_single_token_wide_range():
+    """Token values spread over 60 binades: those more than 23 binades below
+    the largest are rounded in the fixed-point image; the error stays far
+    inside the fp32-order bound, and zeros, subnormal and negative values
+    are handled."""
+    K, N = 4096, 512
+    g = torch.Generator().manual_seed(11)
+    mag = torch.pow(2.0, torch.randint(-40, 20, (1, K), generator=g).float())
+    x = (torch.randn(1, K, generator=g) * mag).to(torch.bfloat16)
+    x[0, :16] = 0.0
+    x[0, 16:20] = torch.tensor([1e-39, -1e-39, 5e-40, -3e-40]).to(torch.bfloat16)  # subnormal
+    q_w = torch.randint(-127, 128, (N, K), dtype=torch.int8, generator=g)
+    s_ch = torch.rand(N, generator=g) * 1e-3 + 1e-5
+    _check_w8a16(x, q_w, s_ch)
+
+
+def test_w8a16_single_token_zero_and_nonfinite():
+    K, N = 1024, 288
+    q_w = torch.randint(-127, 128, (N, K), dtype=torch.int8)
+    s_ch = torch.rand(N) + 0.5
+    y = sq.w8a16_mm(torch.zeros(1, K, dtype=torch.bfloat16).cuda(), q_w.cuda(), s_ch.cuda())
+    assert torch.equal(y.cpu().view(torch.int16), torch.zeros(1, N, dtype=torch.int16))
+    # a token with no fixed-point image (inf or NaN) gives NaN everywhere
+    for bad in (float("inf"), float("nan")):
+        x = inputs.gen_x(1, K, 3)
+        x[0, 500] = bad
+        y = sq.w8a16_mm(x.cuda(), q_w.cuda(), s_ch.cuda()).cpu()
+        assert torch.all(torch.isnan(y.float()))
+    sq.check_device_error()
 
 
 # ----------------------------------------------------------- error codes

@@ -49,10 +49,12 @@ def test_cluster_size_limits():
 def test_long_k_small_m_uses_stream_k():
     # 272 K blocks per tile: whole splits would give 90 per CTA, so every SM
     # takes an equal range of the (tile, K block) space instead
-    for M in (1, 16):
-        p = plan(W8A16, M, 5120, 17408)
-        assert (p["kernel"], p["grid"], p["splits"], p["tile_m"]) == (2, B200_SMS, 0, 16)
-        assert p["workspace_bytes"] == slots_bytes(B200_SMS, 16)
+    p = plan(W8A16, 16, 5120, 17408)
+    assert (p["kernel"], p["grid"], p["splits"], p["tile_m"]) == (2, B200_SMS, 0, 16)
+    assert p["workspace_bytes"] == slots_bytes(B200_SMS, 16)
+    # group-wise scales keep the tensor-core schedule for one token as well
+    p = plan(sq.OP_W8A16_GROUP, 1, 5120, 17408)
+    assert (p["kernel"], p["grid"], p["splits"], p["tile_m"]) == (2, B200_SMS, 0, 16)
     assert plan(W8A8, 8, 5120, 17408)["kernel"] == 2
 
 
@@ -71,8 +73,8 @@ def test_block_scaled_pairs_and_large_m_w8a16():
     # per-group activations x gs128 weights: one CTA per 128 x 128 tile
     p = plan(sq.OP_PG128, 2048, 5120, 5120)
     assert (p["kernel"], p["tile_m"], p["tile_n"], p["grid"]) == (1, 128, 128, B200_SMS)
-    # group-wise W8A16 plans like per-channel W8A16
-    for M in (1, 16, 8192):
+    # group-wise W8A16 plans like per-channel W8A16 from two tokens on
+    for M in (2, 16, 8192):
         assert plan(sq.OP_W8A16_GROUP, M, 5120, 17408) == plan(W8A16, M, 5120, 17408)
     # M > 32: the weights are converted into a bf16 copy in the workspace
     p = plan(W8A16, 8192, 5120, 17408)
@@ -96,3 +98,20 @@ def test_bad_arguments():
         plan(W8A8, 8, 5120, 200)  # K % 128
     with pytest.raises(sq.SqError):
         plan(9, 8, 5120, 5120)
+
+
+def test_single_token_w8a16_runs_as_matrix_vector():
+    # one token, per-channel scales: one contiguous run of rows per CTA on
+    # the CUDA cores, whole K, K / 64 compute threads plus a producer warp
+    p = plan(W8A16, 1, 5120, 17408)
+    assert (p["kernel"], p["grid"], p["tile_m"], p["tile_n"], p["splits"]) == \
+        (5, B200_SMS, 1, -(-5120 // B200_SMS), 1)
+    # fewer rows than SMs: one row per CTA
+    p = plan(W8A16, 1, 16, 128)
+    assert (p["kernel"], p["grid"], p["tile_n"]) == (5, 16, 1)
+    # the widest block (15 compute warps of 64 codes per thread + 1) still
+    # fits; 16 compute warps do not
+    assert plan(W8A16, 1, 144, 30720)["kernel"] == 5
+    assert plan(W8A16, 1, 272, 30848)["kernel"] == 2
+    # two tokens stay on the tensor cores
+    assert plan(W8A16, 2, 5120, 17408)["kernel"] == 2

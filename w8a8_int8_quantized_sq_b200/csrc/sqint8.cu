@@ -10,6 +10,7 @@
 #include "gemm.cuh"
 #include "gemm2.cuh"
 #include "gemm3.cuh"
+#include "gemv.cuh"
 #include "peak.cuh"
 #include "quant.cuh"
 
@@ -486,8 +487,59 @@ sq_status run_gemm(GemmKind kind, const void* act, const void* wt, const float* 
   return SQ_ERR_SHAPE;
 }
 
+// A single token with per-channel scales: the CUDA-core matrix-vector kernel,
+// rows dealt round-robin to at most one CTA per SM, when its threads and
+// shared-memory stages fit.
+bool gemv_plan(int64_t M, int64_t N, int64_t K, int sms, GemvLayout* lo, int* grid) {
+  if (M != 1 || sms <= 0) return false;
+  const int g = N < sms ? static_cast<int>(N) : sms;
+  const GemvLayout l = gemv_layout(N, K, g);
+  if (l.S < 2) return false;
+  if (lo) *lo = l;
+  if (grid) *grid = g;
+  return true;
+}
+
+sq_status launch_gemv(const void* x, const int8_t* q_w, const float* s_ch, void* y, int64_t N,
+                      int64_t K, const GemvLayout& l, int grid, cudaStream_t st, bool pdl) {
+  static std::atomic<int> smem_set[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SQ_ERR_CUDA;
+  if (smem_set[dev].load(std::memory_order_acquire) < l.smem) {
+    if (cudaFuncSetAttribute(w8a16_gemv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             l.smem) != cudaSuccess)
+      return SQ_ERR_CUDA;
+    int cur = smem_set[dev].load();
+    while (cur < l.smem && !smem_set[dev].compare_exchange_weak(cur, l.smem)) {
+    }
+  }
+  const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+  __nv_bfloat16* yb = static_cast<__nv_bfloat16*>(y);
+  const int n = static_cast<int>(N), k = static_cast<int>(K);
+  if (!pdl) {
+    w8a16_gemv_kernel<<<grid, l.nwc * 32 + 32, l.smem, st>>>(xb, q_w, s_ch, yb, n, k, l);
+    return launch_status();
+  }
+  // programmatic dependent launch: the weight stream starts while the
+  // preceding kernel runs; the token is read after griddep_wait
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(l.nwc * 32 + 32);
+  cfg.dynamicSmemBytes = l.smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, w8a16_gemv_kernel, xb, q_w, s_ch, yb, n, k, l) != cudaSuccess)
+    return SQ_ERR_CUDA;
+  return launch_status();
+}
+
 // W8A16 workspace.  M <= 32 (dequant on load): [counter region][stream-K
-// slots].  Larger M: [counter region][bf16 weights N x K].
+// slots] (a single token on the matrix-vector kernel leaves it unused).
+// Larger M: [counter region][bf16 weights N x K].
 size_t w8a16_ws_bytes(int64_t M, int64_t N, int64_t K, int sms, size_t* w_off) {
   if (M <= 32) {
     if (w_off) *w_off = 0;
@@ -698,7 +750,15 @@ sq_status sq_describe_plan(int op, int64_t M, int64_t N, int64_t K, int sms,
   const GemmPlan p = plan_gemm(kind, M, N, K, sms);
   const int tiles = p.tiles_r * p.tiles_c;
   sq_plan_info r{};
-  if (p.pair) {
+  GemvLayout gl{};
+  int ggrid = 0;
+  if (op == SQ_OP_W8A16 && gemv_plan(M, N, K, sms, &gl, &ggrid)) {
+    r.kernel = 5;
+    r.grid = ggrid;
+    r.tile_m = 1;
+    r.tile_n = gl.rows_max;
+    r.splits = 1;
+  } else if (p.pair) {
     r.kernel = 0;
     r.grid = 2 * (tiles < sms / 2 ? tiles : sms / 2);
     r.tile_m = 256;
@@ -806,6 +866,10 @@ sq_status w8a16_mm(const void* x_bf16, const int8_t* q_w, const float* s_ch, voi
   if (!workspace || ws_bytes < need) return SQ_ERR_WORKSPACE;
   if (!aligned16(workspace)) return SQ_ERR_ALIGN;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  GemvLayout gl{};
+  int ggrid = 0;
+  if (gemv_plan(M, N, K, sms, &gl, &ggrid))  // one token: a matrix-vector product
+    return launch_gemv(x_bf16, q_w, s_ch, y_bf16, N, K, gl, ggrid, st, overlap_on());
   if (M <= 32)  // weight-read bound: int8 weights are converted on load, in the GEMM
     return run_gemm(GK_W8A16_CONV, x_bf16, q_w, nullptr, s_ch, nullptr, y_bf16, M, N, K,
                     workspace, ws_bytes, st, overlap_on());
