@@ -127,8 +127,7 @@ __global__ void __launch_bounds__(kGemvMaxThreads, 1)
     *xmax = 0u;
     fence_mbar_init();
   }
-  // this thread's first row scale, requested now and used at the end
-  const float sc0 = t < nrows ? __ldg(s_ch + b + static_cast<size_t>(t) * G) : 1.0f;
+  float sc0 = 1.0f;  // a compute thread's first row scale, used at the end
   __syncthreads();
 
   if (warp == nwc) {
@@ -156,7 +155,8 @@ __global__ void __launch_bounds__(kGemvMaxThreads, 1)
     }
   } else {
     // ------------------------------------------------------ compute warps
-    griddep_wait();  // the token may come from the preceding kernel
+    griddep_wait();  // the token and the scales may come from the preceding kernel
+    if (t < nrows) sc0 = __ldg(s_ch + b + static_cast<size_t>(t) * G);  // requested early
     const int T = nwc * 32;
     const int chunks = K / 16;
     uint4 xr[kGemvChunks][2];  // this thread's 64 token values, bf16
@@ -273,7 +273,7 @@ __global__ void __launch_bounds__(kGemvMaxThreads, 1)
     long long sum = 0;
     for (int w = 0; w < nwc; ++w) sum += part[i * nwc + w];
     const size_t row = static_cast<size_t>(b) + static_cast<size_t>(i) * G;
-    const float sc = i == t ? sc0 : __ldg(s_ch + row);
+    const float sc = (i == t && warp < nwc) ? sc0 : __ldg(s_ch + row);
     const double r = static_cast<double>(sum) * static_cast<double>(sc) * unscale;
     y[row] = finite ? __double2bfloat16(r) : __ushort_as_bfloat16(0x7FC0u);
   }
