@@ -16,9 +16,9 @@
 // summed over lanes and warps in int64, so the dot product is exact and
 // independent of the order; y = bf16(fp64(sum) * s_ch * 2^-sh), two
 // roundings (the fp64 product and the bf16 conversion), like the oracle's
-// fp64 sum times s_ch rounded to bf16.  One dp4a per code per plane: four
-// integer instructions per four codes and plane, against nine for an exact
-// int8-to-fp32 conversion and packed fp32 FMAs.  A token holding inf or NaN
+// fp64 sum times s_ch rounded to bf16.  One dp4a per four codes and plane,
+// so four integer instructions per four codes, against nine for an exact
+// int8-to-fp32 conversion with packed fp32 FMAs.  A token holding inf or NaN
 // has no fixed-point image: every output is then NaN.
 //
 // Rows are dealt to the CTAs round-robin (CTA b takes rows b, b + G, b + 2G,
